@@ -1,0 +1,189 @@
+/*
+ * mala.h -- C ABI of the B200 (sm_100a) MALA attention library.
+ *
+ * MALA (MassAlloc Attention) is causal softmax attention that scores every
+ * legal causal QK tile but skips a tile's post-score work when the tile's
+ * largest per-key contribution ratio falls below tau/Lq, Lq = i + 1 being the
+ * number of causally visible keys of query row i (agihunt.info, "MassAlloc
+ * Attention: Let Attention Allocate Its Own Compute", method paragraphs;
+ * arXiv 2609.32712 abstract on aihot.vn).
+ *
+ * Conventions shared by every call:
+ *   - All tensor arguments are DEVICE pointers to caller-owned, contiguous
+ *     memory on the current CUDA device. Every pointer must be 16-byte
+ *     aligned. The library never allocates device memory.
+ *   - bf16 tensors are passed as void* holding bfloat16 bit patterns.
+ *   - Layouts are BSHD: q, o, dO, dq [B, L, Hq, d]; k, v, dk, dv
+ *     [B, L, Hkv, d]; lse [B, Hq, L] fp32 in natural-log units.
+ *   - Tiles: nq = ceil(L / Bq) query blocks, nk = ceil(L / Bk) key blocks;
+ *     tile (qb, kb) is legal iff kb*Bk <= min((qb+1)*Bq, L) - 1.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream). Arguments are validated on
+ *     the host before anything is enqueued: on any error return nothing is
+ *     written and nothing is launched.
+ *   - GQA: query head hq reads KV head hq / (Hq / Hkv).
+ *   - Supported: d in {64, 128}; Bq == Bk in {64, 128}; any L >= 1 (a ragged
+ *     last tile is fine); B, Hq, Hkv >= 1 with Hq % Hkv == 0.
+ *   - Device-side waits are bounded. If one expires the kernel records
+ *     MALA_ERR_DEVICE_TIMEOUT in a device status word and returns;
+ *     mala_check_status() reports it.
+ *   - Calls are not reentrant with respect to the same output buffers.
+ */
+#ifndef MALA_H_
+#define MALA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MALA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MALA_API __attribute__((visibility("default")))
+#else
+#define MALA_API
+#endif
+
+typedef enum mala_status {
+    MALA_OK = 0,
+    MALA_ERR_INVALID_ARG = 1,    /* null pointer, Hq % Hkv != 0, L < 1, scale <= 0, tau < 0, NaN */
+    MALA_ERR_UNSUPPORTED = 2,    /* d, Bq, Bk outside the supported set; pointer not 16-B aligned */
+    MALA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than the size query returns */
+    MALA_ERR_CUDA = 4,           /* a CUDA runtime / driver call or a launch failed */
+    MALA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait expired (see mala_check_status) */
+} mala_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+MALA_API const char* mala_status_string(int status);
+
+/* MALA_ABI_VERSION of the loaded library. */
+MALA_API int mala_abi_version(void);
+
+/*
+ * mala_fwd -- MALA forward (training / prefill of a whole sequence).
+ *
+ * Source: agihunt.info MALA digest, method paragraphs (forward gate against
+ * the running online-softmax state, conservative per query block, visit
+ * order from the diagonal back, forced first tile, LSE as the saved state).
+ *
+ * For every (b, hq, qb), key blocks kb run from the last legal one down to 0.
+ * Every legal tile is scored, S = scale * Q K^T (bf16 in, fp32 accumulate).
+ * With (m_r, l_r) the online-softmax state over previously kept tiles, the
+ * tile is kept iff it is the block's first legal tile, or tau == 0, or some
+ * row r with a live key satisfies
+ *     max_live_j exp(s_rj - m_r) / l_r >= tau / (i_r + 1)      (ties keep).
+ * A kept tile updates (m, l) and O for every row of the block; a skipped
+ * tile loads no V and does no softmax update and no PV.
+ *
+ *   q        [B, L, Hq, d]  bf16, in
+ *   k, v     [B, L, Hkv, d] bf16, in
+ *   o        [B, L, Hq, d]  bf16, out: O_i = acc_i / l_i
+ *   lse      [B, Hq, L]     fp32, out: LSE_i = m_i + ln l_i (natural log)
+ *   scale    > 0 (usually 1/sqrt(d)); tau >= 0 (tau = 0: full attention)
+ *   kept_tiles [B*Hq] int32, out (required): kept tiles per (b, hq); zeroed
+ *            by the call on `stream` before the kernel accumulates into it
+ *   keep_map   [B, Hq, nq, nk] uint8, out, nullable (test/debug only): 1 for
+ *            a kept tile, 0 for a skipped legal tile; entries of illegal
+ *            tiles are not written. The method itself never reads it.
+ */
+MALA_API int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int L, int d, float scale, float tau, int Bq, int Bk, int32_t* kept_tiles,
+             uint8_t* keep_map, void* stream);
+
+/*
+ * Workspace bytes mala_bwd needs: an fp32 dQ accumulator [B, L, Hq, d] and
+ * an fp32 D = rowsum(dO * O) vector [B, Hq, L], each 256-byte aligned.
+ * Returns 0 for invalid sizes.
+ */
+MALA_API size_t mala_bwd_workspace_size(int B, int Hq, int L, int d);
+
+/*
+ * mala_bwd -- MALA backward.
+ *
+ * Source: agihunt.info MALA digest, method paragraphs (backward gate against
+ * the final normaliser, nested support without a stored mask, approximate
+ * rather than exact gradient).
+ *
+ * Scores are recomputed on every legal tile. A tile is kept iff tau == 0 or
+ * some live (i, j) has exp(s_ij - LSE_i) >= tau / (i + 1); no tile is forced.
+ * With D_i = <dO_i, O_i>, a kept tile computes for its live entries
+ *   P = exp(s - LSE), dP = dO V^T, dS = P * (dP - D),
+ *   dV += P^T dO, dK += scale * dS^T Q, dQ += scale * dS K;
+ * a skipped tile does none of these. dK / dV sum over the GQA group.
+ *
+ *   q, o, dO   [B, L, Hq, d]  bf16, in (o and lse as written by mala_fwd)
+ *   k, v       [B, L, Hkv, d] bf16, in
+ *   lse        [B, Hq, L]     fp32, in
+ *   dq         [B, L, Hq, d]  bf16, out
+ *   dk, dv     [B, L, Hkv, d] bf16, out
+ *   workspace  device scratch of >= mala_bwd_workspace_size(B, Hq, L, d)
+ *              bytes, 256-byte aligned, caller-owned; contents on entry are
+ *              ignored (the call clears what it uses)
+ *   kept_tiles [B*Hq] int32, out (required): backward-kept tiles per (b, hq)
+ *   keep_map   [B, Hq, nq, nk] uint8, out, nullable: as for mala_fwd
+ */
+MALA_API int mala_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int L, int d,
+             float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
+             int32_t* kept_tiles, uint8_t* keep_map, void* stream);
+
+/*
+ * Workspace bytes mala_decode needs for n_splits partial results:
+ * fp32 O partials [B, Hq, n_splits, d] and fp32 LSE partials
+ * [B, Hq, n_splits], each 256-byte aligned. Returns 0 for invalid sizes.
+ */
+MALA_API size_t mala_decode_workspace_size(int B, int Hq, int d, int n_splits);
+
+/*
+ * Deterministic split count mala_decode uses when n_splits == 0: enough
+ * (b, KV head, split) work units to fill the GPU's SMs, at least one tile per
+ * split. Depends only on its arguments and the current device's SM count.
+ */
+MALA_API int mala_decode_default_splits(int B, int Hkv, int Lk, int Bk);
+
+/*
+ * mala_decode -- one new query per sequence against a KV cache of Lk keys.
+ *
+ * Source: agihunt.info MALA digest, method and limitations paragraphs (one
+ * tau for training and serving, the KV cache kept whole, decode speed limited
+ * by cache reads).
+ *
+ * The query is row i = Lk - 1, so every key is visible and Lq = Lk. The nk =
+ * ceil(Lk / Bk) key tiles are cut into contiguous splits of
+ * T = ceil(nk / n_splits) tiles (split s covers [s*T, min((s+1)*T, nk))).
+ * Each split runs the forward gate with its own fresh state from its newest
+ * tile to its oldest, always keeping its newest tile; the partial results
+ * are merged by their LSEs: LSE = log sum_s exp(LSE_s),
+ * O = sum_s exp(LSE_s - LSE) O_s. V of a tile is loaded only if some query
+ * head of the GQA group keeps it.
+ *
+ *   q          [B, Hq, d]       bf16, in
+ *   kcache, vcache [B, Lk, Hkv, d] bf16, in
+ *   o          [B, Hq, d]       bf16, out
+ *   lse        [B, Hq]          fp32, out (natural log)
+ *   n_splits   >= 1, or 0 for mala_decode_default_splits(B, Hkv, Lk, Bk)
+ *   workspace  >= mala_decode_workspace_size(B, Hq, d, n_splits used) bytes
+ *   kept_tiles [B*Hq] int32, out (required): tiles whose PV ran per (b, hq)
+ *   keep_map   [B, Hq, nk] uint8, out, nullable
+ */
+MALA_API int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B,
+                int Hq, int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits,
+                void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
+                void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word. Returns MALA_OK, MALA_ERR_DEVICE_TIMEOUT if any kernel since the last
+ * check gave up on a bounded wait, or MALA_ERR_CUDA if the stream reports an
+ * error.
+ */
+MALA_API int mala_check_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MALA_H_ */

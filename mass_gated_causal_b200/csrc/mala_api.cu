@@ -1,0 +1,186 @@
+// mala_api.cu -- the C ABI declared in include/mala.h.
+//
+// Host side only: argument validation, TMA tensor-map construction, launch
+// configuration. Every step of the computation runs in the kernels included
+// below. The driver's cuTensorMapEncodeTiled is reached through
+// cudaGetDriverEntryPoint, so the library loads on machines without a GPU
+// driver (its symbols can be inspected there) and needs no -lcuda.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mala.h"
+#include "mala_bwd.cuh"
+#include "mala_decode.cuh"
+#include "mala_fwd.cuh"
+
+namespace {
+
+__device__ unsigned int g_mala_status;  // per-device status word, see mala_check_status
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a contiguous bf16 BSHD tensor [B, S, H, D] with a
+// {64, 1, rows, 1} box and 128-byte swizzle: one box is a [rows x 64] tile of
+// one head, 128 bytes per row, the layout the UMMA descriptors expect.
+bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int D, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                           static_cast<cuuint64_t>(S) * H * D * 2};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+unsigned* status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_mala_status) != cudaSuccess) return nullptr;
+  return static_cast<unsigned*>(p);
+}
+
+int check_train_shape(int B, int Hq, int Hkv, int L, int d, float scale, float tau, int Bq, int Bk) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1) return MALA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return MALA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return MALA_ERR_INVALID_ARG;
+  if (!(tau >= 0.f) || !std::isfinite(tau)) return MALA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if (Bq != Bk || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
+  // element counts must fit the int arithmetic of the kernels
+  if (static_cast<long long>(B) * L * Hq * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq >= (1ll << 24)) return MALA_ERR_UNSUPPORTED;
+  return MALA_OK;
+}
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? MALA_OK
+             : MALA_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- forward
+template <int D, int BK, bool G>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+               const mala::FwdParams& p, cudaStream_t st) {
+  using Lay = mala::FwdLayout<D, BK>;
+  auto kern = mala::mala_fwd_kernel<D, BK, G>;
+  if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.n_super) * p.B * p.Hq;
+  kern<<<grid, 192, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mo, p);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
+template <int D, int BK>
+int launch_fwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const CUtensorMap& mo, const mala::FwdParams& p, cudaStream_t st) {
+  return gate ? launch_fwd<D, BK, true>(mq, mk, mv, mo, p, st) : launch_fwd<D, BK, false>(mq, mk, mv, mo, p, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mala_status_string(int status) {
+  switch (status) {
+    case MALA_OK: return "MALA_OK";
+    case MALA_ERR_INVALID_ARG: return "MALA_ERR_INVALID_ARG";
+    case MALA_ERR_UNSUPPORTED: return "MALA_ERR_UNSUPPORTED";
+    case MALA_ERR_WORKSPACE: return "MALA_ERR_WORKSPACE";
+    case MALA_ERR_CUDA: return "MALA_ERR_CUDA";
+    case MALA_ERR_DEVICE_TIMEOUT: return "MALA_ERR_DEVICE_TIMEOUT";
+    default: return "MALA_ERR_UNKNOWN";
+  }
+}
+
+int mala_abi_version(void) { return MALA_ABI_VERSION; }
+
+int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int L,
+             int d, float scale, float tau, int Bq, int Bk, int32_t* kept_tiles, uint8_t* keep_map,
+             void* stream) {
+  if (!q || !k || !v || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return MALA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_bshd_map(&mq, q, B, L, Hq, d, 128) || !make_bshd_map(&mk, k, B, L, Hkv, d, Bk) ||
+      !make_bshd_map(&mv, v, B, L, Hkv, d, Bk) || !make_bshd_map(&mo, o, B, L, Hq, d, 128))
+    return MALA_ERR_CUDA;
+  unsigned* status = status_ptr();
+  if (!status) return MALA_ERR_CUDA;
+  mala::FwdParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
+  p.nq = (L + Bq - 1) / Bq;
+  p.nk = (L + Bk - 1) / Bk;
+  p.n_super = (L + 127) / 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;
+  p.lse = lse;
+  p.kept_tiles = kept_tiles;
+  p.keep_map = keep_map;
+  p.status = status;
+  if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
+  const bool gate = tau > 0.f;
+  if (d == 128 && Bk == 128) return launch_fwd_gate<128, 128>(gate, mq, mk, mv, mo, p, st);
+  if (d == 64 && Bk == 128) return launch_fwd_gate<64, 128>(gate, mq, mk, mv, mo, p, st);
+  if (d == 128 && Bk == 64) return launch_fwd_gate<128, 64>(gate, mq, mk, mv, mo, p, st);
+  return launch_fwd_gate<64, 64>(gate, mq, mk, mv, mo, p, st);
+}
+
+size_t mala_bwd_workspace_size(int, int, int, int) { return 0; }
+int mala_bwd(const void*, const void*, const void*, const void*, const void*, const float*, void*, void*, void*,
+             int, int, int, int, int, float, float, int, int, void*, size_t, int32_t*, uint8_t*, void*) {
+  return MALA_ERR_UNSUPPORTED;
+}
+size_t mala_decode_workspace_size(int, int, int, int) { return 0; }
+int mala_decode_default_splits(int, int, int, int) { return 1; }
+int mala_decode(const void*, const void*, const void*, void*, float*, int, int, int, int, int, float, float, int,
+                int, void*, size_t, int32_t*, uint8_t*, void*) {
+  return MALA_ERR_UNSUPPORTED;
+}
+
+int mala_check_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MALA_ERR_CUDA;
+  unsigned int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_mala_status, sizeof(h)) != cudaSuccess) return MALA_ERR_CUDA;
+  if (h != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_mala_status, &zero, sizeof(zero)) != cudaSuccess) return MALA_ERR_CUDA;
+    return MALA_ERR_DEVICE_TIMEOUT;
+  }
+  return MALA_OK;
+}
+
+}  // extern "C"

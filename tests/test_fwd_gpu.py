@@ -1,0 +1,82 @@
+"""MALA forward on the GPU (C ABI mala_fwd) against the fp64 oracle.
+
+Element-wise comparisons on seeded inputs at sizes the oracle finishes in
+seconds: several tiles, a ragged last tile, GQA, both tile sizes, tau = 0
+(full attention) and tau > 0. Rules and tolerances are in tests/parity.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import (LSE_ABS, O_REL_L2, compare_fwd_decisions, illegal_untouched, rel_l2)
+from workloads import C0, C1, C1_IID, TrainWorkload, bf16_bits_to_f64, make_train_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _to_dev(bits):
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _to_f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def run_fwd_case(mala, w, tau, L=None):
+    L = w.L if L is None else L
+    inp = make_train_inputs(w, L=L)
+    q, k, v = (_to_dev(inp[x]) for x in ("q", "k", "v"))
+    o, lse, kept, km = mala.forward(q, k, v, w.scale, tau, w.Bq, w.Bk, keep_map=True)
+    assert mala.mala_check_status() == 0
+    torch.cuda.synchronize()
+    qf, kf, vf = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v"))
+    ref = oracle.fwd(qf, kf, vf, w.scale, tau, w.Bq, w.Bk)
+    km_h = km.cpu().numpy()
+    assert illegal_untouched(km_h, L, w.Bq, w.Bk)
+    dec = compare_fwd_decisions(km_h, ref["keep"], ref["margin"], L, w.Bq, w.Bk)
+    assert dec["bad"] == 0, dec["bad_sites"][:10]
+    assert dec["in_margin"] + dec["cascaded"] <= max(2, dec["compared"] // 1000), dec
+    kept_h = kept.cpu().numpy()
+    assert (kept_h == (km_h == 1).reshape(kept_h.shape[0], -1).sum(1)).all()
+    e_o = rel_l2(_to_f64(o), ref["o"])
+    e_lse = float(np.abs(lse.cpu().numpy().astype(np.float64) - ref["lse"]).max())
+    assert e_o <= O_REL_L2, e_o
+    assert e_lse <= LSE_ABS, e_lse
+    if tau == 0:
+        assert (km_h == 1).sum() == (ref["keep"] == 1).sum()
+    print(f"[fwd parity] L={L} d={w.d} H={w.Hq}/{w.Hkv} B={w.Bq} tau={tau}: o_rel_l2={e_o:.3e} "
+          f"lse_abs={e_lse:.3e} tiles={dec['compared']} in_margin={dec['in_margin']} cascaded={dec['cascaded']} "
+          f"kept={int(kept_h.sum())}")
+    return {"o_rel_l2": e_o, "lse_abs": e_lse, **{k_: v_ for k_, v_ in dec.items() if k_ != "diverged_blocks"}}
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+def test_fwd_c0(cuda_lib, tau):
+    run_fwd_case(cuda_lib, C0, tau)
+
+
+@pytest.mark.parametrize("L,d,Hq,Hkv,Bt,tau", [
+    (1000, 128, 4, 2, 128, 1.0),   # ragged last tile, GQA
+    (1000, 128, 4, 2, 128, 0.0),
+    (777, 64, 2, 1, 64, 1.0),      # two query blocks per CTA, ragged, GQA
+    (300, 128, 2, 2, 64, 0.5),
+    (129, 64, 3, 3, 128, 4.0),     # one row past a tile boundary
+    (1, 128, 2, 1, 128, 1.0),      # a single row
+    (64, 128, 1, 1, 64, 1.0),
+])
+def test_fwd_small_shapes(cuda_lib, L, d, Hq, Hkv, Bt, tau):
+    w = TrainWorkload("small", 1, Hq, Hkv, L, d, Bt, Bt, seed=3000 + L + d)
+    run_fwd_case(cuda_lib, w, tau)
+
+
+def test_fwd_batch2(cuda_lib):
+    w = TrainWorkload("batch2", 2, 4, 4, 640, 128, 128, 128, seed=3101)
+    run_fwd_case(cuda_lib, w, 1.0)
+
+
+@pytest.mark.parametrize("w,tau", [(C1, 0.0), (C1, 1.0), (C1_IID, 0.0), (C1_IID, 1.0)])
+def test_fwd_c1(cuda_lib, w, tau):
+    run_fwd_case(cuda_lib, w, tau)
