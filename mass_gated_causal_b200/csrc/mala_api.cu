@@ -10,6 +10,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -106,6 +107,26 @@ int launch_fwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, con
   return gate ? launch_fwd<D, BK, true>(mq, mk, mv, mo, p, st) : launch_fwd<D, BK, false>(mq, mk, mv, mo, p, st);
 }
 
+// --------------------------------------------------------------- backward
+template <int D, int BK, bool G>
+int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+               const CUtensorMap& mdk, const CUtensorMap& mdv, const mala::BwdParams& p, cudaStream_t st) {
+  using Lay = mala::BwdLayout<D>;
+  auto kern = mala::mala_bwd_kernel<D, BK, G>;
+  if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.n_super) * p.B * p.Hkv;
+  kern<<<grid, 192, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, p);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
+template <int D, int BK>
+int launch_bwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
+                    const mala::BwdParams& p, cudaStream_t st) {
+  return gate ? launch_bwd<D, BK, true>(mq, mk, mv, mdo, mdk, mdv, p, st)
+              : launch_bwd<D, BK, false>(mq, mk, mv, mdo, mdk, mdv, p, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -158,10 +179,71 @@ int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   return launch_fwd_gate<64, 64>(gate, mq, mk, mv, mo, p, st);
 }
 
-size_t mala_bwd_workspace_size(int, int, int, int) { return 0; }
-int mala_bwd(const void*, const void*, const void*, const void*, const void*, const float*, void*, void*, void*,
-             int, int, int, int, int, float, float, int, int, void*, size_t, int32_t*, uint8_t*, void*) {
-  return MALA_ERR_UNSUPPORTED;
+size_t mala_bwd_workspace_size(int B, int Hq, int L, int d) {
+  if (B < 1 || Hq < 1 || L < 1 || (d != 64 && d != 128)) return 0;
+  return align256(static_cast<size_t>(B) * L * Hq * d * 4) + align256(static_cast<size_t>(B) * Hq * L * 4);
+}
+
+int mala_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int L, int d, float scale, float tau, int Bq,
+             int Bk, void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
+             void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return MALA_ERR_UNSUPPORTED;
+  const size_t need = mala_bwd_workspace_size(B, Hq, L, d);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  if (!make_bshd_map(&mq, q, B, L, Hq, d, 128) || !make_bshd_map(&mk, k, B, L, Hkv, d, 128) ||
+      !make_bshd_map(&mv, v, B, L, Hkv, d, 128) || !make_bshd_map(&mdo, dO, B, L, Hq, d, 128) ||
+      !make_bshd_map(&mdk, dk, B, L, Hkv, d, 128) || !make_bshd_map(&mdv, dv, B, L, Hkv, d, 128))
+    return MALA_ERR_CUDA;
+  unsigned* status = status_ptr();
+  if (!status) return MALA_ERR_CUDA;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         align256(static_cast<size_t>(B) * L * Hq * d * 4));
+  mala::BwdParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
+  p.nq = (L + Bq - 1) / Bq;
+  p.nk = (L + Bk - 1) / Bk;
+  p.n_super = (L + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;
+  p.lse = lse;
+  p.dvec = dvec;
+  p.dq_acc = dq_acc;
+  p.kept_tiles = kept_tiles;
+  p.keep_map = keep_map;
+  p.status = status;
+
+  const long long chunks = static_cast<long long>(B) * L * Hq * (d / 8);  // 16-byte chunks of O / dO
+  const int pre_grid = static_cast<int>(std::min<long long>((chunks + 255) / 256, 148LL * 16));
+  if (d == 128)
+    mala::mala_bwd_pre_kernel<128><<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(o),
+        static_cast<const uint4*>(dO), dvec, reinterpret_cast<float4*>(dq_acc), kept_tiles, B, L, Hq);
+  else
+    mala::mala_bwd_pre_kernel<64><<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(o),
+        static_cast<const uint4*>(dO), dvec, reinterpret_cast<float4*>(dq_acc), kept_tiles, B, L, Hq);
+  if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
+
+  const bool gate = tau > 0.f;
+  if (d == 128 && Bk == 128) rc = launch_bwd_gate<128, 128>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
+  else if (d == 64 && Bk == 128) rc = launch_bwd_gate<64, 128>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
+  else if (d == 128 && Bk == 64) rc = launch_bwd_gate<128, 64>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
+  else rc = launch_bwd_gate<64, 64>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
+  if (rc != MALA_OK) return rc;
+
+  const long long n8 = static_cast<long long>(B) * L * Hq * d / 8;
+  const int cv_grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
+  mala::mala_dq_convert_kernel<<<cv_grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
+                                                         static_cast<uint4*>(dq), n8);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 size_t mala_decode_workspace_size(int, int, int, int) { return 0; }
 int mala_decode_default_splits(int, int, int, int) { return 1; }

@@ -1,2 +1,567 @@
+// mala_bwd.cuh -- MALA backward kernels for sm_100a.
+//
+// Method (agihunt.info, "MassAlloc Attention: Let Attention Allocate Its Own
+// Compute", method paragraphs): the backward recomputes the scores of every
+// legal tile and tests each tile against the FINAL log-normaliser written by
+// the forward -- keep iff some live (i, j) has exp(s_ij - LSE_i) >= tau/(i+1)
+// -- with no stored mask and no forced tile. A skipped tile does no
+// probability reconstruction, no dP, dS, dQ, dK or dV.
+//
+// Kernels:
+//   mala_bwd_pre_kernel   D_i = <dO_i, O_i>, clears the fp32 dQ accumulator
+//                         and the per-head counters
+//   mala_bwd_kernel       dK/dV-stationary main loop (below)
+//   mala_dq_convert_kernel fp32 dQ accumulator -> bf16 dQ
+//
+// mala_bwd_kernel: one CTA owns 128 keys (one key block when Bk = 128, two
+// when Bk = 64) of one (b, KV head) and walks the query tiles of every query
+// head of the GQA group, 128 queries at a time, from the diagonal tile to the
+// end. dK and dV accumulate in TMEM across the whole walk.
+//   warps 0-3  thread t owns key row t (TMEM lane t of S^T, dP^T, dK, dV) and,
+//              for the dQ drain, query row t of the tile (TMEM lane t of dQ)
+//   warp  4    producer: K, V once; Q tiles and the per-query LSE / threshold
+//              / D vectors through a 2-stage ring
+//   warp  5    MMA issuer: S^T = K Q^T, then for kept tiles the dO TMA,
+//              dP^T = V dO^T, dV += P^T dO, dK += dS^T Q, dQ = dS K
+// P^T and dS^T share one shared-memory tile: dS^T overwrites P^T once the dV
+// MMA that reads P^T has finished. dQ reuses the dP^T TMEM columns and is
+// added to the fp32 accumulator with vector reductions.
 #pragma once
+
 #include "mala_ptx.cuh"
+
+namespace mala {
+
+struct BwdParams {
+  int B, Hq, Hkv, L, G;
+  int nq, nk, n_super;
+  float scale, scale_log2, log2_tau;
+  const float* lse;   // [B, Hq, L]
+  const float* dvec;  // [B, Hq, L]: D_i
+  float* dq_acc;      // [B, L, Hq, d] fp32
+  int32_t* kept_tiles;
+  uint8_t* keep_map;
+  unsigned* status;
+};
+
+constexpr uint32_t kBwdAny = 1u << 4;
+constexpr uint32_t kBwdAbort = 1u << 5;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int T_BYTES = 128 * D * 2;  // a 128-row tile of K, V, Q or dO
+  static constexpr int PS_BYTES = 128 * 128 * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + T_BYTES;
+  static constexpr int OFF_Q = OFF_V + T_BYTES;  // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * T_BYTES;
+  static constexpr int OFF_PS = OFF_DO + T_BYTES;
+  static constexpr int OFF_VEC = OFF_PS + PS_BYTES;  // [2 stages][LSE2, T, D][128] fp32
+  static constexpr int OFF_BAR = OFF_VEC + 2 * 3 * 128 * 4;
+  // kv_full, q_full[2], q_empty[2], s_full, st_free, dec, do_full, do_empty,
+  // dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free, ps_free, mma_final
+  static constexpr int N_BARS = 18;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int BYTES = OFF_MISC + 64;
+  static constexpr int ALLOC_BYTES = BYTES + 1024;
+  static constexpr int TMEM_COLS = 512;  // S^T 128 | dP^T/dQ 128 | dK D | dV D
+  static_assert(ALLOC_BYTES <= 232448, "backward shared memory exceeds the per-CTA limit");
+};
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D, int BK, bool kGate>
+__global__ void __launch_bounds__(192, 1)
+    mala_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                    const BwdParams p) {
+  using Lay = BwdLayout<D>;
+  constexpr int BQ = BK, QPB = 128 / BQ, KPB = 128 / BK;
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+  constexpr uint32_t IDESC_KN = idesc_bf16(128, D, false, true);  // A K-major, B MN-major
+  constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, true, true);   // A, B MN-major
+  constexpr int TB = Lay::T_BYTES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem + Lay::OFF_K;
+  uint8_t* sV = smem + Lay::OFF_V;
+  uint8_t* sQ = smem + Lay::OFF_Q;
+  uint8_t* sDO = smem + Lay::OFF_DO;
+  uint8_t* sPS = smem + Lay::OFF_PS;
+  float* sVec = reinterpret_cast<float*>(smem + Lay::OFF_VEC);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;   // [2]
+  uint64_t* q_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* st_free = bars + 6;
+  uint64_t* dec_bar = bars + 7;
+  uint64_t* do_full = bars + 8;
+  uint64_t* do_empty = bars + 9;
+  uint64_t* dp_full = bars + 10;
+  uint64_t* p_ready = bars + 11;
+  uint64_t* dv_done = bars + 12;
+  uint64_t* ds_ready = bars + 13;
+  uint64_t* dq_full = bars + 14;
+  uint64_t* dq_free = bars + 15;
+  uint64_t* ps_free = bars + 16;
+  uint64_t* mma_final = bars + 17;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  uint32_t* tmem_slot = misc + 0;
+  int* abort_flag = reinterpret_cast<int*>(misc + 1);
+  uint32_t* dec_flags = misc + 2;
+  uint32_t* vote = misc + 4;   // [2][4]
+  uint32_t* evote = misc + 12; // [4]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nbk = p.B * p.Hkv;
+  const int bk = blockIdx.x % nbk;
+  const int ks = static_cast<int>(blockIdx.x / nbk);  // ascending: longest walks first
+  const int b = bk / p.Hkv, hkv = bk % p.Hkv;
+  const int k0 = ks * 128;
+  const int nqs = p.n_super - ks;
+  const int T = p.G * nqs;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 33);  // expect_tx arrival + 32 vector-writing lanes
+      mbar_init(&q_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(st_free, 128);
+    mbar_init(dec_bar, 1);
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(dv_done, 1);
+    mbar_init(ds_ready, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(ps_free, 1);
+    mbar_init(mma_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, Lay::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const FailState fs{abort_flag, p.status};
+  const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 256 + D;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * TB);
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_4d(&tm_k, kv_full, sK + h * 16384, h * 64, hkv, k0, b);
+        tma_load_4d(&tm_v, kv_full, sV + h * 16384, h * 64, hkv, k0, b);
+      }
+    }
+    int issued = 0;
+    for (int t = 0; t < T; ++t) {
+      const int st = t & 1;
+      if (t >= 2 && !mbar_wait_warp(&q_empty[st], ((t >> 1) - 1) & 1, fs)) break;
+      const int hq = hkv * p.G + t / nqs;
+      const int i0 = (ks + t % nqs) * 128;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&q_full[st], TB);
+        for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_q, &q_full[st], sQ + st * TB + h * 16384, h * 64, hq, i0, b);
+      }
+      float* vec = sVec + st * 384;
+      const size_t rowbase = static_cast<size_t>(b * p.Hq + hq) * p.L;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = lane * 4 + e;
+        const int i = i0 + r;
+        const bool ok = i < p.L;
+        const float lse2 = ok ? p.lse[rowbase + i] * 1.4426950408889634f : INFINITY;
+        vec[r] = lse2;
+        vec[128 + r] = kGate ? lse2 + p.log2_tau - lg2_approx(static_cast<float>(i + 1)) : 0.f;
+        vec[256 + r] = ok ? p.dvec[rowbase + i] : 0.f;
+      }
+      mbar_arrive(&q_full[st]);
+      issued = t + 1;
+    }
+    if (lane == 0) {
+      mbar_wait_drain(kv_full, 0);
+      for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait_drain(&q_full[t & 1], (t >> 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
+      const uint32_t sPSa = smem_u32(sPS);
+      int nd = 0;
+      bool ok = mbar_wait(kv_full, 0, fs);
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t & 1;
+        const int hq = hkv * p.G + t / nqs;
+        const int i0 = (ks + t % nqs) * 128;
+        const uint32_t sQs = sQa + st * TB;
+        if (!mbar_wait(&q_full[st], (t >> 1) & 1, fs)) break;
+        if (t >= 1 && !mbar_wait(st_free, (t - 1) & 1, fs)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16_ss(tS, sdesc_sw128(sKa + off, 16, 1024), sdesc_sw128(sQs + off, 16, 1024), IDESC_S,
+                       kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        if (!mbar_wait(dec_bar, t & 1, fs)) break;
+        const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(dec_flags);
+        if (dec & kBwdAbort) break;
+        if (dec & kBwdAny) {
+          if (nd >= 1 && !mbar_wait(do_empty, (nd - 1) & 1, fs)) break;
+          mbar_arrive_expect_tx(do_full, TB);
+          for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, i0, b);
+          if (nd >= 1 && !mbar_wait(dq_free, (nd - 1) & 1, fs)) break;
+          if (!mbar_wait(do_full, nd & 1, fs)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_bf16_ss(tDP, sdesc_sw128(sVa + off, 16, 1024), sdesc_sw128(sDOa + off, 16, 1024), IDESC_S,
+                         kk > 0 ? 1u : 0u);
+          }
+          umma_commit(dp_full);
+          if (!mbar_wait(p_ready, nd & 1, fs)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO
+            const uint64_t a = sdesc_sw128(sPSa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sDOa + kk * 2048, 16384, 1024);
+            umma_bf16_ss(tDV, a, bd, IDESC_KN, (nd > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(do_empty);
+          umma_commit(dv_done);
+          if (!mbar_wait(ds_ready, nd & 1, fs)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q
+            const uint64_t a = sdesc_sw128(sPSa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sQs + kk * 2048, 16384, 1024);
+            umma_bf16_ss(tDK, a, bd, IDESC_KN, (nd > 0 || kk > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K (dS read MN-major from the dS^T tile)
+            const uint64_t a = sdesc_sw128(sPSa + kk * 2048, 16384, 1024);
+            const uint64_t bd = sdesc_sw128(sKa + kk * 2048, 16384, 1024);
+            umma_bf16_ss(tDP, a, bd, IDESC_DQ, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(dq_full);
+          umma_commit(ps_free);
+          ++nd;
+        }
+        umma_commit(&q_empty[st]);
+      }
+      umma_commit(mma_final);
+      if (nd >= 1) mbar_wait_drain(do_full, (nd - 1) & 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ compute warps
+    const int tid = threadIdx.x;
+    const int kj = k0 + tid;  // my key
+    const int ki = tid / BK;  // my key block inside the CTA
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t sPSa = smem_u32(sPS);
+    const float sl2 = p.scale_log2;
+    int nd = 0;
+    bool local_abort = false, all_abort = false;
+    uint32_t r[32];
+
+    for (int t = 0; t < T; ++t) {
+      const int st = t & 1;
+      const int hq = hkv * p.G + t / nqs;
+      const int qs = ks + t % nqs;
+      const int i0 = qs * 128;
+      const bool diag = qs == ks;
+      const float* vec = sVec + st * 384;
+      const bool ok = mbar_wait_warp(s_full, t & 1, fs);
+      local_abort |= !ok;
+      tc_fence_after();
+      uint32_t kbits = 0;
+      if (kGate) {
+        if (ok) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            tmem_ld32(tS + lane_base + ch * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 th = *reinterpret_cast<const float4*>(vec + 128 + ch * 32 + j4 * 4);
+              const float tv[4] = {th.x, th.y, th.z, th.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int il = ch * 32 + j4 * 4 + e;
+                const bool live = !diag || (i0 + il >= kj);
+                if (live && __uint_as_float(r[j4 * 4 + e]) * sl2 >= tv[e]) kbits |= 1u << (il / BQ);
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int qi = 0; qi < QPB; ++qi) {
+          const int qb = qs * QPB + qi, kb = ks * KPB + ki;
+          if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) kbits |= 1u << qi;
+        }
+      }
+      uint32_t wv = 0;
+#pragma unroll
+      for (int qi = 0; qi < QPB; ++qi) wv |= (__ballot_sync(0xffffffffu, (kbits >> qi) & 1u) ? 1u : 0u) << qi;
+      if (lane == 0) vote[(t & 1) * 4 + warp] = wv | (local_abort ? 8u : 0u);
+      named_bar_sync(1, 128);
+      uint32_t kept = 0;  // bit (qi * 2 + ki): sub-tile kept
+      bool any_abort = false;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t vw = vote[(t & 1) * 4 + w];
+        any_abort |= (vw & 8u) != 0;
+        const int kw = (w * 32) / BK;
+#pragma unroll
+        for (int qi = 0; qi < QPB; ++qi)
+          if ((vw >> qi) & 1u) kept |= 1u << (qi * 2 + kw);
+      }
+      if (tid == 0) {
+        *dec_flags = kept | (kept ? kBwdAny : 0u) | (any_abort ? kBwdAbort : 0u);
+        mbar_arrive(dec_bar);
+      }
+      if (any_abort) {
+        all_abort = true;
+        break;
+      }
+      if (tid == 0) {
+        int cnt = 0;
+        for (int qi = 0; qi < QPB; ++qi)
+          for (int kx = 0; kx < KPB; ++kx) {
+            const int qb = qs * QPB + qi, kb = ks * KPB + kx;
+            if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) {
+              const int kp = (kept >> (qi * 2 + kx)) & 1u;
+              if (p.keep_map) p.keep_map[(static_cast<size_t>(b * p.Hq + hq) * p.nq + qb) * p.nk + kb] = kp;
+              cnt += kp;
+            }
+          }
+        if (cnt) atomicAdd(&p.kept_tiles[b * p.Hq + hq], cnt);
+      }
+      if (!kept) {
+        tc_fence_before();
+        mbar_arrive(st_free);
+        continue;
+      }
+      // ---- kept: P^T row of my key, zero outside kept sub-tiles / live entries
+      if (nd >= 1) local_abort |= !mbar_wait_warp(ps_free, (nd - 1) & 1, fs);
+      uint32_t qmask = 0;  // query blocks whose sub-tile with my key block is kept
+#pragma unroll
+      for (int qi = 0; qi < QPB; ++qi) qmask |= ((kept >> (qi * 2 + ki)) & 1u) << qi;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        tmem_ld32(tS + lane_base + ch * 32, r);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int il = ch * 32 + 2 * jj;
+          const bool l0 = ((qmask >> (il / BQ)) & 1u) && (!diag || i0 + il >= kj);
+          const bool l1 = ((qmask >> ((il + 1) / BQ)) & 1u) && (!diag || i0 + il + 1 >= kj);
+          const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(r[2 * jj]), sl2, -vec[il])) : 0.f;
+          const float p1 = l1 ? ex2_approx(fmaf(__uint_as_float(r[2 * jj + 1]), sl2, -vec[il + 1])) : 0.f;
+          pk[jj] = pack_bf16x2(p0, p1);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = ch * 32 + c * 8;
+          st_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pk[4 * c], pk[4 * c + 1],
+                       pk[4 * c + 2], pk[4 * c + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      mbar_arrive(st_free);
+      // ---- dS^T = P^T * (dP^T - D)
+      local_abort |= !mbar_wait_warp(dp_full, nd & 1, fs);
+      tc_fence_after();
+      uint32_t dsp[64];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        tmem_ld32(tDP + lane_base + ch * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = ch * 32 + c * 8;
+          uint32_t pp[4];
+          ld_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pp[0], pp[1], pp[2], pp[3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int il = col + 2 * e;
+            const float d0 = __uint_as_float(r[c * 8 + 2 * e]) - vec[256 + il];
+            const float d1 = __uint_as_float(r[c * 8 + 2 * e + 1]) - vec[256 + il + 1];
+            dsp[ch * 16 + c * 4 + e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * d0, bf16hi_to_f32(pp[e]) * d1);
+          }
+        }
+      }
+      local_abort |= !mbar_wait_warp(dv_done, nd & 1, fs);  // the dV MMA has read P^T
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int col = c * 8;
+        st_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), dsp[4 * c], dsp[4 * c + 1],
+                     dsp[4 * c + 2], dsp[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(ds_ready);
+      // ---- dQ rows of this tile: fp32 reductions into the accumulator
+      local_abort |= !mbar_wait_warp(dq_full, nd & 1, fs);
+      tc_fence_after();
+      {
+        const int i = i0 + tid;
+        float* dst = p.dq_acc + (static_cast<size_t>(b) * p.L + i) * (static_cast<size_t>(p.Hq) * D) +
+                     static_cast<size_t>(hq) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          tmem_ld32(tDP + lane_base + ch * 32, r);
+          tmem_ld_wait();
+          if (i < p.L) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              red_add_v4(dst + ch * 32 + q4 * 4, p.scale * __uint_as_float(r[q4 * 4]),
+                         p.scale * __uint_as_float(r[q4 * 4 + 1]), p.scale * __uint_as_float(r[q4 * 4 + 2]),
+                         p.scale * __uint_as_float(r[q4 * 4 + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+      ++nd;
+    }
+
+    if (!all_abort) {
+      // ---------------------------------------------------------- epilogue
+      const bool okf = mbar_wait_warp(mma_final, 0, fs);
+      tc_fence_after();
+      const uint32_t sQa = smem_u32(sQ);
+      if (okf) {
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t tsrc = (which == 0 ? tDK : tDV) + lane_base;
+          const float mul = which == 0 ? p.scale : 1.f;
+          const uint32_t dst = sQa + which * TB;
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            if (nd > 0) {
+              tmem_ld32(tsrc + ch * 32, r);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) r[j] = 0u;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              pk[jj] = pack_bf16x2(__uint_as_float(r[2 * jj]) * mul, __uint_as_float(r[2 * jj + 1]) * mul);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int col = ch * 32 + c * 8;
+              st_shared_v4(dst + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pk[4 * c], pk[4 * c + 1],
+                           pk[4 * c + 2], pk[4 * c + 3]);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      const unsigned okall = __ballot_sync(0xffffffffu, okf);
+      if (lane == 0) evote[warp] = okall == 0xffffffffu ? 1u : 0u;
+      named_bar_sync(1, 128);
+      if (tid == 0 && (evote[0] & evote[1] & evote[2] & evote[3])) {
+        for (int h = 0; h < D / 64; ++h) {
+          tma_store_4d(&tm_dk, sQ + h * 16384, h * 64, hkv, k0, b);
+          tma_store_4d(&tm_dv, sQ + TB + h * 16384, h * 64, hkv, k0, b);
+        }
+        tma_store_commit_and_wait();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    if (lane == 0) mbar_wait_drain(mma_final, 0);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::TMEM_COLS);
+  }
+}
+
+// D_i = <dO_i, O_i> for every (b, i, hq); clears dq_acc and the counters.
+// 8 elements (16 bytes) per thread; D/8 threads per row.
+template <int D>
+__global__ void __launch_bounds__(256) mala_bwd_pre_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dO,
+                                                          float* __restrict__ dvec, float4* __restrict__ dq_acc,
+                                                          int32_t* __restrict__ kept, int B, int L, int Hq) {
+  constexpr int TPR = D / 8;
+  const long long total = static_cast<long long>(B) * L * Hq * TPR;
+  const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  // the loop bound is taken at the warp's first lane so that every lane of a
+  // warp runs the same iterations (the row reduction shuffles across lanes)
+  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g - lane < total;
+       g += nthreads) {
+    const bool active = g < total;
+    float s = 0.f;
+    if (active) {
+      const uint4 a = o[g];
+      const uint4 c = dO[g];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        s = fmaf(bf16lo_to_f32(av[e]), bf16lo_to_f32(cv[e]), s);
+        s = fmaf(bf16hi_to_f32(av[e]), bf16hi_to_f32(cv[e]), s);
+      }
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off, TPR);
+    if (active) {
+      if ((g % TPR) == 0) {
+        const long long row = g / TPR;  // (b * L + i) * Hq + hq
+        const int hq = static_cast<int>(row % Hq);
+        const long long bi = row / Hq;
+        const int i = static_cast<int>(bi % L);
+        const int bb = static_cast<int>(bi / L);
+        dvec[(static_cast<long long>(bb) * Hq + hq) * L + i] = s;
+      }
+      dq_acc[2 * g] = make_float4(0.f, 0.f, 0.f, 0.f);
+      dq_acc[2 * g + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < B * Hq; i += blockDim.x) kept[i] = 0;
+}
+
+// bf16 dQ from the fp32 accumulator (the softmax scale is already applied).
+__global__ void __launch_bounds__(256) mala_dq_convert_kernel(const float4* __restrict__ acc, uint4* __restrict__ dq,
+                                                             long long n8) {
+  const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < n8; g += nthreads) {
+    const float4 a = acc[2 * g], c = acc[2 * g + 1];
+    dq[g] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+  }
+}
+
+}  // namespace mala
