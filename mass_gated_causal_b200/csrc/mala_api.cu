@@ -127,6 +127,23 @@ int launch_bwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, con
               : launch_bwd<D, BK, false>(mq, mk, mv, mdo, mdk, mdv, p, st);
 }
 
+// ----------------------------------------------------------------- decode
+template <int D, int BK, bool G>
+int launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecParams& p, cudaStream_t st) {
+  using Lay = mala::DecLayout<D, BK>;
+  auto kern = mala::mala_decode_split_kernel<D, BK, G>;
+  if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(p.B) * p.Hkv * p.n_splits;
+  kern<<<grid, 160, Lay::ALLOC_BYTES, st>>>(mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
+template <int D, int BK>
+int launch_dec_gate(bool gate, const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecParams& p,
+                    cudaStream_t st) {
+  return gate ? launch_dec<D, BK, true>(mk, mv, p, st) : launch_dec<D, BK, false>(mk, mv, p, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -245,11 +262,81 @@ int mala_bwd(const void* q, const void* k, const void* v, const void* o, const v
                                                          static_cast<uint4*>(dq), n8);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
-size_t mala_decode_workspace_size(int, int, int, int) { return 0; }
-int mala_decode_default_splits(int, int, int, int) { return 1; }
-int mala_decode(const void*, const void*, const void*, void*, float*, int, int, int, int, int, float, float, int,
-                int, void*, size_t, int32_t*, uint8_t*, void*) {
-  return MALA_ERR_UNSUPPORTED;
+size_t mala_decode_workspace_size(int B, int Hq, int d, int n_splits) {
+  if (B < 1 || Hq < 1 || n_splits < 1 || (d != 64 && d != 128)) return 0;
+  const size_t parts = static_cast<size_t>(B) * Hq * n_splits;
+  return align256(parts * d * 4) + align256(parts * 4);
+}
+
+int mala_decode_default_splits(int B, int Hkv, int Lk, int Bk) {
+  if (B < 1 || Hkv < 1 || Lk < 1 || Bk < 1) return 1;
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    sms = 148;
+  const long long nk = (static_cast<long long>(Lk) + Bk - 1) / Bk;
+  const long long units = static_cast<long long>(B) * Hkv;
+  long long s = (16LL * sms + units - 1) / units;  // about 16 CTAs per SM in total
+  s = std::max(1LL, std::min(s, nk));
+  const long long per = (nk + s - 1) / s;  // every split non-empty
+  s = (nk + per - 1) / per;
+  return static_cast<int>(std::min(s, 65535LL));
+}
+
+int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,
+                int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, void* workspace,
+                size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  if (!q || !kcache || !vcache || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lk < 1 || Hq % Hkv != 0 || n_splits < 0) return MALA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale) || !(tau >= 0.f) || !std::isfinite(tau)) return MALA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > mala::kDecMaxG) return MALA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Lk * Hkv * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, kcache, vcache, o, lse};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return MALA_ERR_UNSUPPORTED;
+  if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk);
+  if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
+  const size_t need = mala_decode_workspace_size(B, Hq, d, n_splits);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mk, mv;
+  if (!make_bshd_map(&mk, kcache, B, Lk, Hkv, d, Bk) || !make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk))
+    return MALA_ERR_CUDA;
+  unsigned* status = status_ptr();
+  if (!status) return MALA_ERR_CUDA;
+  const size_t parts = static_cast<size_t>(B) * Hq * n_splits;
+  mala::DecParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lk = Lk; p.G = Hq / Hkv;
+  p.nk = (Lk + Bk - 1) / Bk;
+  p.n_splits = n_splits;
+  p.tiles_per_split = (p.nk + n_splits - 1) / n_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.thr = tau > 0.f ? std::log2(tau) - std::log2(static_cast<float>(Lk)) : 0.f;
+  p.q = static_cast<const uint16_t*>(q);
+  p.o_part = static_cast<float*>(workspace);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(parts * d * 4));
+  p.kept_tiles = kept_tiles;
+  p.keep_map = keep_map;
+  p.status = status;
+  if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
+  const bool gate = tau > 0.f;
+  int rc;
+  if (d == 128 && Bk == 128) rc = launch_dec_gate<128, 128>(gate, mk, mv, p, st);
+  else if (d == 64 && Bk == 128) rc = launch_dec_gate<64, 128>(gate, mk, mv, p, st);
+  else if (d == 128 && Bk == 64) rc = launch_dec_gate<128, 64>(gate, mk, mv, p, st);
+  else rc = launch_dec_gate<64, 64>(gate, mk, mv, p, st);
+  if (rc != MALA_OK) return rc;
+  const int rows = B * Hq;
+  if (d == 128)
+    mala::mala_decode_combine_kernel<128><<<(rows + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
+                                                                         static_cast<uint16_t*>(o), lse, rows,
+                                                                         n_splits);
+  else
+    mala::mala_decode_combine_kernel<64><<<(rows + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
+                                                                        static_cast<uint16_t*>(o), lse, rows,
+                                                                        n_splits);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
 int mala_check_status(void* stream) {
