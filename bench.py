@@ -1,0 +1,534 @@
+"""MALA benchmark: one JSON line on rank 0.
+
+A step is one MALA training pass of the attention operator -- mala_fwd then
+mala_bwd -- on the 32K GQA workload (B=1, Hq=32, Hkv=8, L=32768, d=128,
+Bq=Bk=128, tau=1) with inputs resident in HBM. The same run also measures
+the library's tau=0 path (full attention) on the same inputs and the decode
+workload (B=8, Lk=131072, Hq=32, Hkv=8, d=128, Bk=128), reported as
+sub-objects of the same line.
+
+  value      effective TFLOP/s, whole job: FLOPs counted as QK over every live
+             causal pair plus post-score matmuls over the live pairs of kept
+             tiles (fwd 2d*N_legal + 2d*N_f, bwd 2d*N_legal + 8d*N_b), summed
+             over ranks, divided by the max-over-ranks device time
+  e2e        the same metric through the C ABI starting from pinned host
+             buffers: H2D of q, k, v, dO and D2H of dq, dk, dv inside the
+             timed region
+  roofline   the dominant kernel's achieved rate against the measured peak
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (a per-GPU
+head slice, as in head-sharded attention); no collective on the data path;
+scaling is weak. `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import C2, C4, WORKLOADS, default_workers  # noqa: E402
+
+METRIC = "MALA fwd+bwd ms & eff. TFLOP/s (% bf16 peak) at 32K/128K, τ=1; retained-tile %"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# --------------------------------------------------------------------------
+# Work accounting (host logic; unit-tested on CPU)
+# --------------------------------------------------------------------------
+def live_pairs(L: int, Bq: int, Bk: int) -> np.ndarray:
+    """[nq, nk] number of live (i, j <= i) pairs of every tile."""
+    nq, nk = -(-L // Bq), -(-L // Bk)
+    out = np.zeros((nq, nk), dtype=np.int64)
+    for qb in range(nq):
+        i = np.arange(qb * Bq, min((qb + 1) * Bq, L))
+        for kb in range(nk):
+            j0, j1 = kb * Bk, min((kb + 1) * Bk, L)
+            out[qb, kb] = np.clip(np.minimum(i, j1 - 1) - j0 + 1, 0, None).sum()
+    return out
+
+
+def train_flops(d: int, B: int, Hq: int, L: int, live: np.ndarray, keep_f, keep_b):
+    """Effective FLOPs of one fwd and one bwd (keep maps [B,Hq,nq,nk] or None = all kept)."""
+    n_legal = B * Hq * int(live.sum())
+    n_f = n_legal if keep_f is None else int(((keep_f == 1) * live).sum())
+    n_b = n_legal if keep_b is None else int(((keep_b == 1) * live).sum())
+    return {"n_legal": n_legal, "n_f": n_f, "n_b": n_b,
+            "fwd": 2 * d * n_legal + 2 * d * n_f, "bwd": 2 * d * n_legal + 8 * d * n_b}
+
+
+def decode_bytes(B, Hq, Hkv, Lk, d, Bk, keep_map):
+    """Algorithmic bytes of one decode step: all K, V of tiles kept by >= 1 head of
+    the group, q in and o out (bf16)."""
+    nk = -(-Lk // Bk)
+    rows = np.array([min((t + 1) * Bk, Lk) - t * Bk for t in range(nk)], dtype=np.int64)
+    G = Hq // Hkv
+    if keep_map is None:
+        v_tiles = np.ones((B, Hkv, nk), dtype=bool)
+    else:
+        v_tiles = (keep_map.reshape(B, Hkv, G, nk) == 1).any(axis=2)
+    k_all = B * Lk * Hkv * d * 2
+    v_kept = int((v_tiles * rows[None, None, :]).sum()) * d * 2
+    return {"k_all": k_all, "v_kept": v_kept, "qo": 2 * B * Hq * d * 2, "total": k_all + v_kept + 2 * B * Hq * d * 2,
+            "v_tile_frac": float(v_tiles.mean())}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------------
+# Clock sampling during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# CUDA arm
+# --------------------------------------------------------------------------
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_cuda(args):
+    import torch
+    import mass_gated_causal_b200 as mala
+
+    world, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk = peaks()
+    w = WORKLOADS[args.workload]
+    tau = 1.0
+    workers = default_workers()
+    t_gen = time.time()
+    from workloads import make_train_inputs
+    inp = make_train_inputs(w, workers=workers)
+    t_gen = time.time() - t_gen
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v, do = (to_dev(inp[x]) for x in ("q", "k", "v", "do"))
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    stream = torch.cuda.current_stream(dev)
+    # outputs and workspace allocated once
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    kept_f = torch.empty((B * Hq,), dtype=torch.int32, device=dev)
+    kept_b = torch.empty((B * Hq,), dtype=torch.int32, device=dev)
+    ws_bytes = mala.mala_bwd_workspace_size(B, Hq, L, d)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    nq, nk = -(-L // w.Bq), -(-L // w.Bk)
+
+    def step(tau_, km_f=None, km_b=None):
+        rc = mala.mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, kept_f, km_f, stream)
+        assert rc == 0, mala.mala_status_string(rc)
+        rc = mala.mala_bwd(q, k, v, o, do, lse, dq, dk, dv, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, ws,
+                           ws_bytes, kept_b, km_b, stream)
+        assert rc == 0, mala.mala_status_string(rc)
+
+    # one diagnostic pass with keep maps: retained tiles and the FLOP count
+    live = live_pairs(L, w.Bq, w.Bk)
+    km_f = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8, device=dev)
+    km_b = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8, device=dev)
+    step(tau, km_f, km_b)
+    assert mala.mala_check_status(stream) == 0
+    kmf, kmb = km_f.cpu().numpy(), km_b.cpu().numpy()
+    fl = train_flops(d, B, Hq, L, live, kmf, kmb)
+    fl0 = train_flops(d, B, Hq, L, live, None, None)
+    legal = (live > 0)
+    kept_frac_f = (kmf == 1).reshape(B * Hq, -1).sum(1) / legal.sum()
+    kept_frac_b = (kmb == 1).reshape(B * Hq, -1).sum(1) / legal.sum()
+    del km_f, km_b
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1, e2 in ev:
+            e0.record(stream)
+            fn(e1)
+            e2.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        tot = [e0.elapsed_time(e2) for e0, e1, e2 in ev]
+        first = [e0.elapsed_time(e1) for e0, e1, e2 in ev]
+        second = [e1.elapsed_time(e2) for e0, e1, e2 in ev]
+        return tot, first, second
+
+    def train_step(tau_):
+        def fn(mid=None):
+            rc = mala.mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, kept_f, None, stream)
+            assert rc == 0
+            if mid is not None:
+                mid.record(stream)
+            rc = mala.mala_bwd(q, k, v, o, do, lse, dq, dk, dv, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, ws,
+                               ws_bytes, kept_b, None, stream)
+            assert rc == 0
+        return fn
+
+    gpu_id = str(local)
+    try:
+        props = torch.cuda.get_device_properties(dev)
+        if getattr(props, "uuid", None) is not None:
+            u = str(props.uuid)
+            gpu_id = u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+
+    with ClockSampler(gpu_id) as clk:
+        tot1, f1, b1 = timed(train_step(tau), args.steps, args.warmup)
+    clocks = clk.summary()
+    assert mala.mala_check_status(stream) == 0
+    ms = max_over_ranks(float(np.mean(tot1)))
+    ms_f = max_over_ranks(float(np.mean(f1)))
+    ms_b = max_over_ranks(float(np.mean(b1)))
+    step_flops = fl["fwd"] + fl["bwd"]
+    value = world * step_flops / (ms * 1e-3) / 1e12
+
+    # tau = 0 (full attention) on the same inputs
+    tot0, f0, b0 = timed(train_step(0.0), max(2, args.steps // 2), max(3, args.warmup // 2))
+    ms0 = max_over_ranks(float(np.mean(tot0)))
+    ms0_f = max_over_ranks(float(np.mean(f0)))
+    ms0_b = max_over_ranks(float(np.mean(b0)))
+    flops0 = fl0["fwd"] + fl0["bwd"]
+
+    # e2e through the C ABI from pinned host buffers
+    hq_, hk_, hv_, hdo_ = (torch.from_numpy(inp[x].view(np.int16)).view(torch.bfloat16).pin_memory()
+                           for x in ("q", "k", "v", "do"))
+    hdq = torch.empty(dq.shape, dtype=torch.bfloat16).pin_memory()
+    hdk = torch.empty(dk.shape, dtype=torch.bfloat16).pin_memory()
+    hdv = torch.empty(dv.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * 2 for t in (hq_, hk_, hv_, hdo_))
+    d2h = sum(t.numel() * 2 for t in (hdq, hdk, hdv))
+
+    def e2e_fn(mid=None):
+        q.copy_(hq_, non_blocking=True)
+        k.copy_(hk_, non_blocking=True)
+        v.copy_(hv_, non_blocking=True)
+        do.copy_(hdo_, non_blocking=True)
+        train_step(tau)(mid)
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    tote, _, _ = timed(e2e_fn, max(2, args.steps // 2), 1)
+    ms_e2e = max_over_ranks(float(np.mean(tote)))
+
+    # decode workload
+    dec = None
+    if not args.no_decode:
+        dec = run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world)
+
+    # roofline of the dominant kernel (fwd or bwd call, timed with events on its stream)
+    peak_t = pk["bf16_tflops_sustained"]
+    t_fwd = fl["fwd"] / (ms_f * 1e-3) / 1e12
+    t_bwd = fl["bwd"] / (ms_b * 1e-3) / 1e12
+    dom = "mala_bwd_kernel" if ms_b >= ms_f else "mala_fwd_kernel"
+    ach = t_bwd if dom == "mala_bwd_kernel" else t_fwd
+    roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peak_t, "unit": "TFLOP/s",
+            "frac": round(ach / peak_t, 4), "traffic": args.traffic,
+            "peak_kind": f"bf16 dense, {pk['source']} sustained",
+            "timed_unit": "mala_bwd call (pre + main + dq convert kernels)" if dom == "mala_bwd_kernel"
+            else "mala_fwd call (one kernel)",
+            "fwd": {"ms": round(ms_f, 3), "tflops": round(t_fwd, 2), "frac": round(t_fwd / peak_t, 4)},
+            "bwd": {"ms": round(ms_b, 3), "tflops": round(t_bwd, 2), "frac": round(t_bwd / peak_t, 4)}}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(w, inp, tau, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded structured generator)",
+        "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "L": L, "d": d, "Bq": w.Bq, "Bk": w.Bk,
+                   "tau": tau, "scale": w.scale, "seed": w.seed, "parallelism": f"replicas x{world} (head slices)",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "frac_of_peak": round(value / world / peak_t, 4),
+        "retained_tiles": {"fwd_mean": round(float(kept_frac_f.mean()), 4),
+                           "fwd_min": round(float(kept_frac_f.min()), 4),
+                           "fwd_max": round(float(kept_frac_f.max()), 4),
+                           "bwd_mean": round(float(kept_frac_b.mean()), 4),
+                           "bwd_min": round(float(kept_frac_b.min()), 4),
+                           "bwd_max": round(float(kept_frac_b.max()), 4),
+                           "live_pair_frac_fwd": round(fl["n_f"] / fl["n_legal"], 4),
+                           "live_pair_frac_bwd": round(fl["n_b"] / fl["n_legal"], 4)},
+        "fwd_ms": round(ms_f, 3), "bwd_ms": round(ms_b, 3), "step_tflop": round(step_flops / 1e12, 3),
+        "fullattn_tau0": {"ms_per_step": round(ms0, 3), "fwd_ms": round(ms0_f, 3), "bwd_ms": round(ms0_b, 3),
+                          "tflops": round(world * flops0 / (ms0 * 1e-3) / 1e12, 3),
+                          "frac_of_peak": round(flops0 / (ms0 * 1e-3) / 1e12 / peak_t, 4),
+                          "mala_speedup": round(ms0 / ms, 3)},
+        "e2e": {"value": round(world * step_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": roof,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "peaks": pk,
+        "input_gen_s": round(t_gen, 1),
+    }
+    if dec is not None:
+        line["decode"] = dec
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world):
+    from workloads import make_decode_inputs
+    w = C4
+    inp = make_decode_inputs(w, workers=workers)
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, kc, vc = (to_dev(inp[x]) for x in ("q", "kcache", "vcache"))
+    B, Hq, d = q.shape
+    Lk, Hkv = kc.shape[1], kc.shape[2]
+    ns = mala.mala_decode_default_splits(B, Hkv, Lk, w.Bk)
+    nk = -(-Lk // w.Bk)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    kept = torch.empty((B * Hq,), dtype=torch.int32, device=dev)
+    wsb = mala.mala_decode_workspace_size(B, Hq, d, ns)
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+    out = {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "Lk": Lk, "d": d, "Bk": w.Bk, "n_splits": ns}
+    for tau in (1.0, 0.0):
+        km = torch.zeros((B, Hq, nk), dtype=torch.uint8, device=dev)
+        rc = mala.mala_decode(q, kc, vc, o, lse, B, Hq, Hkv, Lk, d, w.scale, tau, w.Bk, ns, ws, wsb, kept, km, stream)
+        assert rc == 0
+        assert mala.mala_check_status(stream) == 0
+        kmh = km.cpu().numpy()
+        by = decode_bytes(B, Hq, Hkv, Lk, d, w.Bk, kmh)
+        del km
+
+        def fn(mid=None, tau_=tau):
+            rc_ = mala.mala_decode(q, kc, vc, o, lse, B, Hq, Hkv, Lk, d, w.scale, tau_, w.Bk, ns, ws, wsb, kept, None,
+                                   stream)
+            assert rc_ == 0
+            if mid is not None:
+                mid.record(stream)
+        tot, _, _ = timed(fn, max(5, args.steps * 2), max(3, args.warmup))
+        us = max_over_ranks(float(np.median(tot))) * 1e3
+        gbs = by["total"] / (us * 1e-6) / 1e9
+        out[f"tau{int(tau)}"] = {"us_per_step": round(us, 1), "us_per_token": round(us / B, 2),
+                                 "GBps": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
+                                 "bytes_per_step": by["total"], "v_tile_frac": round(by["v_tile_frac"], 4),
+                                 "retained_tile_frac_per_head": round(float((kmh == 1).mean()), 4)}
+    out["mala_speedup"] = round(out["tau0"]["us_per_step"] / out["tau1"]["us_per_step"], 3)
+    out["hbm_peak_gbs"] = pk["hbm_gbs"]
+    return out
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline leg and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample(w, inp, tau, n_blocks, seed):
+    """Seeded sample of query blocks; the timed oracle work is forward of those
+    blocks plus the dQ part of their backward."""
+    rng = np.random.default_rng(seed)
+    nq = -(-w.L // w.Bq)
+    qb = rng.choice(nq, size=min(n_blocks, nq * w.B * w.Hq), replace=True)
+    hq = rng.integers(0, w.Hq, size=qb.shape[0])
+    b = rng.integers(0, w.B, size=qb.shape[0])
+    return [(int(x), int(y), int(z)) for x, y, z in zip(b, hq, qb)]
+
+
+def run_oracle_sample(w, qf, kf, vf, dof, tau, sel):
+    import oracle
+    live = live_pairs(w.L, w.Bq, w.Bk)
+    t0 = time.perf_counter()
+    f = oracle.fwd(qf, kf, vf, w.scale, tau, w.Bq, w.Bk, sel=sel, with_margin=False)
+    o = np.nan_to_num(f["o"])
+    lse = np.nan_to_num(f["lse"])
+    g = oracle.bwd(qf, kf, vf, o, dof, lse, w.scale, tau, w.Bq, w.Bk, selq=sel, selk=[], with_margin=False)
+    dt = time.perf_counter() - t0
+    flops = 0
+    for (b, h, qb) in sel:
+        row_live = live[qb]
+        nf = int(((f["keep"][b, h, qb] == 1) * row_live).sum())
+        nbk = int(((g["keep"][b, h, qb] == 1) * row_live).sum())
+        nl = int(row_live.sum())
+        flops += (2 * w.d * nl + 2 * w.d * nf) + (2 * w.d * nl + 4 * w.d * nbk)  # fwd + (QK, dP, dQ)
+    return flops, dt
+
+
+def cpu_baseline(w, inp, tau, seconds):
+    import oracle
+    from workloads import bf16_bits_to_f64
+    qf, kf, vf, dof = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v", "do"))
+    n = 4
+    flops = dt = 0.0
+    # grow the sample until it costs about `seconds` of host time
+    while True:
+        sel = oracle_sample(w, inp, tau, n, seed=w.seed + 500)
+        flops, dt = run_oracle_sample(w, qf, kf, vf, dof, tau, sel)
+        if dt >= seconds / 4 or n >= 4096:
+            break
+        n *= 2
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{len(sel)} seeded query blocks of {w.name}: forward + dQ part of "
+                                        f"the backward, {flops / 1e9:.1f} GFLOP effective in {dt:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from workloads import bf16_bits_to_f64, make_train_inputs
+    w = WORKLOADS[args.workload]
+    tau = 1.0
+    inp = make_train_inputs(w, workers=default_workers())
+    qf, kf, vf, dof = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v", "do"))
+    n = max(4, args.ref_blocks)
+    for i in range(args.warmup):
+        run_oracle_sample(w, qf, kf, vf, dof, tau, oracle_sample(w, inp, tau, 2, seed=w.seed + 900 + i))
+    times, fl = [], []
+    for s in range(args.steps):
+        sel = oracle_sample(w, inp, tau, n, seed=w.seed + 1000 + s)
+        f, dt = run_oracle_sample(w, qf, kf, vf, dof, tau, sel)
+        times.append(dt)
+        fl.append(f)
+    value = sum(fl) / sum(times) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(times)), 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded structured generator)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d, "Bq": w.Bq,
+                       "Bk": w.Bk, "tau": tau},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: {n} seeded query blocks of {w.name}, forward + dQ part "
+                                       f"of the backward"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("cuda", "reference"), default="cuda")
+    ap.add_argument("--workload", default=C2.name, choices=sorted(k for k, v in WORKLOADS.items() if hasattr(v, "L")))
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--ref-blocks", type=int, default=16)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture (reported as is)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "cuda":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,51 @@
+"""Host-side accounting of the benchmark (FLOPs, bytes), checked on the CPU."""
+import numpy as np
+
+import bench
+
+
+def test_live_pairs_sum_is_causal_triangle():
+    for L, Bt in ((1024, 64), (1000, 128), (777, 64), (1, 128), (129, 128)):
+        lp = bench.live_pairs(L, Bt, Bt)
+        assert lp.sum() == L * (L + 1) // 2
+        # brute force on the tile grid
+        i = np.arange(L)[:, None]
+        j = np.arange(L)[None, :]
+        live = (j <= i).astype(np.int64)
+        nq = -(-L // Bt)
+        for qb in range(nq):
+            for kb in range(nq):
+                assert lp[qb, kb] == live[qb * Bt:(qb + 1) * Bt, kb * Bt:(kb + 1) * Bt].sum()
+
+
+def test_train_flops_tau0_conventions():
+    d, B, Hq, L = 128, 1, 4, 1000
+    lp = bench.live_pairs(L, 128, 128)
+    f = bench.train_flops(d, B, Hq, L, lp, None, None)
+    n = B * Hq * L * (L + 1) // 2
+    assert f["fwd"] == 4 * d * n
+    assert f["bwd"] == 10 * d * n
+    keep = np.zeros((B, Hq) + lp.shape, dtype=np.uint8)
+    g = bench.train_flops(d, B, Hq, L, lp, keep, keep)
+    assert g["fwd"] == 2 * d * n and g["bwd"] == 2 * d * n
+
+
+def test_decode_bytes():
+    B, Hq, Hkv, Lk, d, Bk = 2, 8, 2, 1000, 128, 128
+    nk = -(-Lk // Bk)
+    full = bench.decode_bytes(B, Hq, Hkv, Lk, d, Bk, None)
+    assert full["k_all"] == B * Lk * Hkv * d * 2
+    assert full["v_kept"] == full["k_all"]
+    km = np.zeros((B, Hq, nk), dtype=np.uint8)
+    km[0, 5, 3] = 1  # KV head 1 of batch 0, tile 3
+    one = bench.decode_bytes(B, Hq, Hkv, Lk, d, Bk, km)
+    assert one["v_kept"] == Bk * d * 2
+    km[0, 4, 3] = 1  # same group, same tile: V still loaded once
+    assert bench.decode_bytes(B, Hq, Hkv, Lk, d, Bk, km)["v_kept"] == Bk * d * 2
+    km[0, 4, nk - 1] = 1  # ragged last tile
+    assert bench.decode_bytes(B, Hq, Hkv, Lk, d, Bk, km)["v_kept"] == (Bk + Lk - (nk - 1) * Bk) * d * 2
+
+
+def test_peaks_present():
+    p = bench.peaks()
+    assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
