@@ -175,6 +175,30 @@ MALA_API int mala_decode(const void* q, const void* kcache, const void* vcache, 
                 void* stream);
 
 /*
+ * mala_decode_noalloc -- mala_decode without a caller-provided workspace.
+ *
+ * The operator papers have no counterpart to this call: it exists for
+ * callers that cannot allocate device memory, for example a plugin inside a
+ * host engine that owns all device memory and offers it no allocator, or a
+ * serving loop that cannot afford the device-wide synchronisation a
+ * cudaMalloc may bring. The call allocates nothing; its split partials live
+ * in one fixed, file-scope device array of mala_decode_noalloc_max_bytes()
+ * bytes (8 MiB) that every GPU loading the library holds until exit.
+ *
+ * Arguments, layouts and results are those of mala_decode, minus the
+ * workspace. A problem whose partials need more than the fixed array
+ * (mala_decode_workspace_size(B, Hq, d, n_splits used) > 8 MiB) returns
+ * MALA_ERR_WORKSPACE and launches nothing. The first call on a device looks
+ * up the array's device address for that device (so make that first call
+ * before any stream capture). All calls share the array: calls that overlap
+ * on the GPU race and must be serialised by the caller.
+ */
+MALA_API size_t mala_decode_noalloc_max_bytes(void);
+MALA_API int mala_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* o, float* lse,
+                                 int B, int Hq, int Hkv, int Lk, int d, float scale, float tau, int Bk,
+                                 int n_splits, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's status
  * word. Returns MALA_OK, MALA_ERR_DEVICE_TIMEOUT if any kernel since the last
  * check gave up on a bounded wait, or MALA_ERR_CUDA if the stream reports an

@@ -33,7 +33,8 @@ MALA_ERR_CUDA = 4
 MALA_ERR_DEVICE_TIMEOUT = 5
 
 EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_bwd_workspace_size", "mala_bwd",
-            "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_check_status")
+            "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_noalloc_max_bytes",
+            "mala_decode_noalloc", "mala_check_status")
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _lib.mala_status_string.argtypes = [_i]
@@ -53,6 +54,9 @@ _lib.mala_decode_default_splits.restype = _i
 _lib.mala_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp,
                              _vp]
 _lib.mala_decode.restype = _i
+_lib.mala_decode_noalloc_max_bytes.restype = _sz
+_lib.mala_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _vp, _vp]
+_lib.mala_decode_noalloc.restype = _i
 _lib.mala_check_status.argtypes = [_vp]
 _lib.mala_check_status.restype = _i
 
@@ -124,6 +128,17 @@ def mala_decode(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_
     return int(_lib.mala_decode(_p(q), _p(kcache), _p(vcache), _p(o), _p(lse), B, Hq, Hkv, Lk, d, float(scale),
                                 float(tau), Bk, n_splits, _p(workspace), int(workspace_bytes), _p(kept_tiles),
                                 _p(keep_map), _stream(stream)))
+
+
+def mala_decode_noalloc_max_bytes() -> int:
+    return int(_lib.mala_decode_noalloc_max_bytes())
+
+
+def mala_decode_noalloc(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, kept_tiles,
+                        keep_map=None, stream=None) -> int:
+    return int(_lib.mala_decode_noalloc(_p(q), _p(kcache), _p(vcache), _p(o), _p(lse), B, Hq, Hkv, Lk, d,
+                                        float(scale), float(tau), Bk, n_splits, _p(kept_tiles), _p(keep_map),
+                                        _stream(stream)))
 
 
 def mala_check_status(stream=None) -> int:

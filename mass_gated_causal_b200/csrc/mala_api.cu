@@ -353,3 +353,112 @@ int mala_check_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.
+//
+// mala_decode_noalloc is mala_decode for callers that cannot allocate device
+// memory: for example a plugin running inside a host engine that owns all
+// device memory and offers it no allocator, or a serving loop that cannot
+// afford the device-wide synchronisation a cudaMalloc may bring. Instead of
+// a caller-provided workspace it uses the file-scope array below, which every
+// GPU that loads this library holds until the process exits. The call itself
+// allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+//
+// The array's name is only a host-side stand-in in host code; its device
+// address is looked up with cudaGetSymbolAddress the first time the entry
+// point runs on a device (with that device current) and cached per device.
+// That first call should therefore come before any stream capture.
+//
+// All calls share the array and it keeps the last call's contents. Every
+// call overwrites all of the split partials it reads (empty splits included),
+// so nothing has to be cleared between calls; calls whose execution overlaps
+// on the GPU race on the array and must be serialised by the caller.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(8) << 20;  // 8 MiB
+__device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device (set-up on first use).
+void* decode_scratch_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mala_decode_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
+
+int mala_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,
+                        int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, int32_t* kept_tiles,
+                        uint8_t* keep_map, void* stream) {
+  if (!q || !kcache || !vcache || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lk < 1 || Hq % Hkv != 0 || n_splits < 0) return MALA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale) || !(tau >= 0.f) || !std::isfinite(tau)) return MALA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > mala::kDecMaxG) return MALA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Lk * Hkv * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, kcache, vcache, o, lse};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return MALA_ERR_UNSUPPORTED;
+  if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk);
+  if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
+  const size_t need = mala_decode_workspace_size(B, Hq, d, n_splits);
+  if (need == 0 || need > kNoAllocScratchBytes) return MALA_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* scratch = decode_scratch_current_device();
+  if (scratch == nullptr) return MALA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap mk, mv;
+  if (!make_bshd_map(&mk, kcache, B, Lk, Hkv, d, Bk) || !make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk))
+    return MALA_ERR_CUDA;
+  unsigned* status = status_ptr();
+  if (!status) return MALA_ERR_CUDA;
+  const size_t parts = static_cast<size_t>(B) * Hq * n_splits;
+  mala::DecParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lk = Lk; p.G = Hq / Hkv;
+  p.nk = (Lk + Bk - 1) / Bk;
+  p.n_splits = n_splits;
+  p.tiles_per_split = (p.nk + n_splits - 1) / n_splits;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.thr = tau > 0.f ? std::log2(tau) - std::log2(static_cast<float>(Lk)) : 0.f;
+  p.q = static_cast<const uint16_t*>(q);
+  p.o_part = static_cast<float*>(scratch);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + align256(parts * d * 4));
+  p.kept_tiles = kept_tiles;
+  p.keep_map = keep_map;
+  p.status = status;
+  if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
+  const bool gate = tau > 0.f;
+  int rc;
+  if (d == 128 && Bk == 128) rc = launch_dec_gate<128, 128>(gate, mk, mv, p, st);
+  else if (d == 64 && Bk == 128) rc = launch_dec_gate<64, 128>(gate, mk, mv, p, st);
+  else if (d == 128 && Bk == 64) rc = launch_dec_gate<128, 64>(gate, mk, mv, p, st);
+  else rc = launch_dec_gate<64, 64>(gate, mk, mv, p, st);
+  if (rc != MALA_OK) return rc;
+  const int rows = B * Hq;
+  if (d == 128)
+    mala::mala_decode_combine_kernel<128><<<(rows + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
+                                                                         static_cast<uint16_t*>(o), lse, rows,
+                                                                         n_splits);
+  else
+    mala::mala_decode_combine_kernel<64><<<(rows + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
+                                                                        static_cast<uint16_t*>(o), lse, rows,
+                                                                        n_splits);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
+}  // extern "C"
