@@ -508,6 +508,52 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_case(args):
+    """One op on a small case (inputs still larger than L2), for ncu captures:
+    fwd / bwd: B=1, Hq=Hkv=16, L=16384, d=128, tau=1; decode: B=8, Lk=32768,
+    Hq=32, Hkv=8, d=128. Runs warmup + steps calls and prints the mean ms."""
+    import torch
+    import mass_gated_causal_b200 as mala
+    from workloads import TrainWorkload, DecodeWorkload, make_decode_inputs, make_train_inputs
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    if args.kernel in ("fwd", "bwd"):
+        w = TrainWorkload("prof_L16k_h16_d128", 1, 16, 16, 16384, 128, 128, 128, seed=1001)
+        inp = make_train_inputs(w, workers=default_workers())
+        q, k, v, do = (to_dev(inp[x]) for x in ("q", "k", "v", "do"))
+        o, lse, _, _ = mala.forward(q, k, v, w.scale, 1.0, w.Bq, w.Bk)
+        if args.kernel == "fwd":
+            def fn():
+                mala.forward(q, k, v, w.scale, 1.0, w.Bq, w.Bk)
+        else:
+            ws = torch.empty((mala.mala_bwd_workspace_size(1, 16, 16384, 128),), dtype=torch.uint8, device=dev)
+
+            def fn():
+                mala.backward(q, k, v, o, do, lse, w.scale, 1.0, w.Bq, w.Bk, workspace=ws)
+    else:
+        w = DecodeWorkload("prof_decode_B8_Lk32k", 8, 32, 8, 32768, 128, 128, seed=1004)
+        inp = make_decode_inputs(w, workers=default_workers())
+        q, kc, vc = (to_dev(inp[x]) for x in ("q", "kcache", "vcache"))
+
+        def fn():
+            mala.decode(q, kc, vc, w.scale, 1.0, w.Bk)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert mala.mala_check_status() == 0
+    print(json.dumps({"kernel_case": args.kernel, "workload": w.name, "ms_mean": e0.elapsed_time(e1) / args.steps}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,12 +565,16 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-blocks", type=int, default=16)
+    ap.add_argument("--kernel", choices=("fwd", "bwd", "decode"), default=None,
+                    help="run one op on a small case (for profiler captures) instead of the benchmark")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture (reported as is)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "cuda":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.kernel is not None:
+        run_kernel_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_cuda(args)
