@@ -128,20 +128,29 @@ int launch_bwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, con
 }
 
 // ----------------------------------------------------------------- decode
-template <int D, int BK, bool G>
+template <int D, int BK, int GP, bool G>
 int launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecParams& p, cudaStream_t st) {
-  using Lay = mala::DecLayout<D, BK>;
-  auto kern = mala::mala_decode_split_kernel<D, BK, G>;
+  using Lay = mala::DecLayout<D, BK, GP>;
+  auto kern = mala::mala_decode_split_kernel<D, BK, GP, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hkv * p.n_splits;
-  kern<<<grid, 160, Lay::ALLOC_BYTES, st>>>(mk, mv, p);
+  kern<<<grid, 288, Lay::ALLOC_BYTES, st>>>(mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
+// GQA group size padded to the next power of two (1, 2, 4, 8).
+template <int D, int BK, bool G>
+int launch_dec_g(const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecParams& p, cudaStream_t st) {
+  if (p.G <= 1) return launch_dec<D, BK, 1, G>(mk, mv, p, st);
+  if (p.G <= 2) return launch_dec<D, BK, 2, G>(mk, mv, p, st);
+  if (p.G <= 4) return launch_dec<D, BK, 4, G>(mk, mv, p, st);
+  return launch_dec<D, BK, 8, G>(mk, mv, p, st);
 }
 
 template <int D, int BK>
 int launch_dec_gate(bool gate, const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecParams& p,
                     cudaStream_t st) {
-  return gate ? launch_dec<D, BK, true>(mk, mv, p, st) : launch_dec<D, BK, false>(mk, mv, p, st);
+  return gate ? launch_dec_g<D, BK, true>(mk, mv, p, st) : launch_dec_g<D, BK, false>(mk, mv, p, st);
 }
 
 }  // namespace

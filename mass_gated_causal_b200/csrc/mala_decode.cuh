@@ -8,17 +8,20 @@
 //
 // Decode reads the whole K cache once per step, so it is bound by HBM
 // bandwidth, not by arithmetic: the dot products run on the CUDA cores and
-// the work is organised around streaming K tiles through shared memory.
+// the kernel is organised around keeping K and V streaming.
 //
 // mala_decode_split_kernel: one CTA per (b, KV head, split). The split's key
 // tiles run newest -> oldest with a fresh online-softmax state per query
 // head; the newest tile of the split is always kept.
-//   warps 0-3  thread j scores key j of the tile against the G query heads
-//              of the GQA group; head gates; P; PV with thread c owning
-//              output column c of every head
-//   warp  4    TMA producer of K tiles through an NK-stage ring
-// V of a tile is requested (by TMA, thread 0) only after the gate has found
-// a head that keeps it. Each split writes (O_s, LSE_s) per head.
+//   warps 0-7  compute: for QK, thread t scores key t % BK against half of the
+//              GQA group's query heads; thread t < G also runs head t's gate
+//   warp  8    TMA producer of K tiles through an NK-stage ring
+// The gate chain (QK, max, gate, normaliser update) never waits for V: the
+// state (m, l) follows from the scores alone. A kept tile's V TMA is issued
+// at its gate, its probabilities and rescale factors go to a ring, and its PV
+// runs kLag kept tiles later, when V has had time to land. PV maps thread t to
+// an output column pair and a quarter of the keys; the quarters are summed at
+// the end of the split. Each split writes (O_s, LSE_s) per head.
 //
 // mala_decode_combine_kernel: LSE = log sum_s exp(LSE_s),
 // O = sum_s exp(LSE_s - LSE) O_s, one warp per (b, query head).
@@ -29,6 +32,7 @@
 namespace mala {
 
 constexpr int kDecMaxG = 8;  // query heads per KV head handled by one CTA
+constexpr int kDecLag = 2;   // kept tiles between a tile's gate and its PV
 
 struct DecParams {
   int B, Hq, Hkv, Lk, G, nk, n_splits, tiles_per_split;
@@ -42,42 +46,54 @@ struct DecParams {
   unsigned* status;
 };
 
-template <int D, int BK>
+template <int D, int BK, int GP>
 struct DecLayout {
-  static constexpr int NK = 4;
-  static constexpr int NV = 2;
+  static constexpr int NK = 3;
+  static constexpr int NV = kDecLag + 1;
+  static constexpr int NP = kDecLag + 1;
+  static constexpr int NT = 256;  // compute threads
   static constexpr int T_BYTES = BK * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * T_BYTES;
-  static constexpr int OFF_Q = OFF_V + NV * T_BYTES;          // fp32 [G][D]
-  static constexpr int OFF_P = OFF_Q + kDecMaxG * D * 4;        // fp32 [G][BK]
-  static constexpr int OFF_RED = OFF_P + kDecMaxG * BK * 4;     // fp32 [4][G]
-  static constexpr int OFF_HEAD = OFF_RED + 4 * kDecMaxG * 4;   // per head: keep, m, alpha
-  static constexpr int OFF_BAR = OFF_HEAD + 4 * kDecMaxG * 4;
-  static constexpr int N_BARS = 2 * NK + NV;                    // k_full, k_empty, v_full
+  static constexpr int OFF_Q = OFF_V + NV * T_BYTES;        // fp32 [GP][D]
+  static constexpr int OFF_P = OFF_Q + GP * D * 4;            // fp32 [NP][BK][GP]
+  static constexpr int OFF_ALPHA = OFF_P + NP * BK * GP * 4;  // fp32 [NP][GP]
+  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [8 warps][GP]
+  static constexpr int OFF_RSUM = OFF_RMAX + 8 * GP * 4;      // fp32 [8 warps][GP]
+  static constexpr int OFF_HEAD = OFF_RSUM + 8 * GP * 4;      // keep, m, l per head
+  static constexpr int OFF_BAR = OFF_HEAD + 3 * GP * 4;
+  static constexpr int N_BARS = 2 * NK + NV;                  // k_full, k_empty, v_full
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
+  static constexpr int ORED_BYTES = 4 * GP * D * 4;           // end-of-split reduction, reuses the K ring
+  static_assert(ORED_BYTES <= NK * T_BYTES, "reduction buffer must fit in the K ring");
   static_assert(ALLOC_BYTES <= 232448, "decode shared memory exceeds the per-CTA limit");
 };
 
-template <int D, int BK, bool kGate>
-__global__ void __launch_bounds__(160, 1)
+template <int D, int BK, int GP, bool kGate>
+__global__ void __launch_bounds__(288, 1)
     mala_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                              const DecParams p) {
-  using Lay = DecLayout<D, BK>;
-  constexpr int NK = Lay::NK, NV = Lay::NV, TB = Lay::T_BYTES;
+  using Lay = DecLayout<D, BK, GP>;
+  constexpr int NK = Lay::NK, NV = Lay::NV, NP = Lay::NP, TB = Lay::T_BYTES, NT = Lay::NT;
+  constexpr int NGRP = NT / BK;                  // QK thread groups (one key per thread per group)
+  constexpr int HPG = (GP + NGRP - 1) / NGRP;    // query heads scored per thread
+  constexpr int WPG = BK / 32;                   // warps per group
+  constexpr int KQ = BK / 4;                     // keys per PV quarter
+  static_assert(D == 128 || D == 64, "head dim");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + Lay::OFF_K;
   uint8_t* sV = smem + Lay::OFF_V;
   float* sq = reinterpret_cast<float*>(smem + Lay::OFF_Q);
-  float* sp = reinterpret_cast<float*>(smem + Lay::OFF_P);
-  float* sred = reinterpret_cast<float*>(smem + Lay::OFF_RED);
-  float* skeep = reinterpret_cast<float*>(smem + Lay::OFF_HEAD);  // 1.0 if head keeps the tile
-  float* smuse = skeep + kDecMaxG;                               // exponent offset (log2 units)
-  float* salpha = smuse + kDecMaxG;                              // rescale factor of O
-  float* sl = salpha + kDecMaxG;                                 // running normaliser
+  float* sP = reinterpret_cast<float*>(smem + Lay::OFF_P);
+  float* sAlpha = reinterpret_cast<float*>(smem + Lay::OFF_ALPHA);
+  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);
+  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);
+  float* sKeep = reinterpret_cast<float*>(smem + Lay::OFF_HEAD);
+  float* sM = sKeep + GP;  // exponent offset per head (log2 units)
+  float* sL = sM + GP;     // running normaliser per head
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + NK;
@@ -108,191 +124,247 @@ __global__ void __launch_bounds__(160, 1)
   }
 
   if (tid == 0) {
-    for (int i = 0; i < NK; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 128); }
+    for (int i = 0; i < NK; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], NT); }
     for (int i = 0; i < NV; ++i) mbar_init(&v_full[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int i = tid; i < G * D; i += blockDim.x) {
+  for (int i = tid; i < GP * D; i += blockDim.x) {
     const int g = i / D, c = i % D;
-    const uint32_t bits = p.q[(static_cast<size_t>(b) * p.Hq + hq0 + g) * D + c];
-    sq[g * D + c] = __uint_as_float(bits << 16);
+    float x = 0.f;
+    if (g < G) x = __uint_as_float(static_cast<uint32_t>(p.q[(static_cast<size_t>(b) * p.Hq + hq0 + g) * D + c]) << 16);
+    sq[g * D + c] = x;
   }
-  if (tid < kDecMaxG) {
-    smuse[tid] = -INFINITY;
-    sl[tid] = 0.f;
+  if (tid < GP) {
+    sM[tid] = -INFINITY;
+    sL[tid] = 0.f;
+    sKeep[tid] = 0.f;  // padded heads (G < GP) never keep
   }
+  for (int i = tid; i < 8 * GP; i += blockDim.x) sRsum[i] = 0.f;
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
       for (int t = 0; t < T; ++t) {
         const int st = t % NK;
         if (t >= NK && !mbar_wait(&k_empty[st], ((t / NK) - 1) & 1, fs)) break;
-        const int kb = t1 - 1 - t;
         mbar_arrive_expect_tx(&k_full[st], TB);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(&tm_k, &k_full[st], sK + st * TB + h * (BK * 128), h * 64, hkv, kb * BK, b);
+          tma_load_4d(&tm_k, &k_full[st], sK + st * TB + h * (BK * 128), h * 64, hkv, (t1 - 1 - t) * BK, b);
         issued = t + 1;
       }
       for (int t = max(0, issued - NK); t < issued; ++t) mbar_wait_drain(&k_full[t % NK], (t / NK) & 1);
     }
     __syncwarp();
-    return;  // the compute warps below use only named barrier 1
+    return;  // the compute warps below synchronise with named barrier 1 only
   }
 
   // ---------------------------------------------------------- compute warps
   const float c2 = p.scale_log2;
-  float acc[kDecMaxG];  // O[g][tid] (thread tid owns output column tid)
+  const int kj = tid % BK;        // QK: my key within the tile
+  const int hbase = (tid / BK) * HPG;  // QK: first of my heads
+  const int cp = tid & 63;        // PV: my output column pair (D = 128) / column (D = 64, cp < 32 pairs)
+  const int kq = tid >> 6;        // PV: my quarter of the keys
+  float acc[GP][2];
 #pragma unroll
-  for (int g = 0; g < kDecMaxG; ++g) acc[g] = 0.f;
-  int my_cnt = 0;  // tiles kept by head tid (threads tid < G)
-  int nv = 0;  // V loads issued (tiles kept by some head)
+  for (int g = 0; g < GP; ++g) acc[g][0] = acc[g][1] = 0.f;
+  int my_cnt = 0;   // tiles kept by head tid (threads tid < G)
+  int nkept = 0;    // kept tiles so far (V loads issued)
+  int ndone = 0;    // kept tiles whose PV has run
   const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+  bool aborted = false;
+
+  auto run_pv = [&](int n) {  // PV of the n-th kept tile (all compute threads)
+    const int vs = n % NV, ps = n % NP;
+    const bool okv = mbar_wait_warp(&v_full[vs], (n / NV) & 1, fs);
+    if (okv && 2 * cp < D) {
+      float al[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) al[g] = sAlpha[ps * GP + g];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) { acc[g][0] *= al[g]; acc[g][1] *= al[g]; }
+      const int col = 2 * cp;
+      const uint32_t vb = sVa + vs * TB + (col >> 6) * (BK * 128) + ((col & 7) << 1);
+      const uint32_t chunk = (col & 63) >> 3;
+      const float* prow = sP + ps * BK * GP;
+#pragma unroll 4
+      for (int jj = 0; jj < KQ; ++jj) {
+        const int j = kq * KQ + jj;
+        uint32_t v2;
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v2) : "r"(vb + j * 128 + ((chunk ^ (j & 7)) << 4)));
+        const float v0 = bf16lo_to_f32(v2), v1 = bf16hi_to_f32(v2);
+        float pr[GP];
+#pragma unroll
+        for (int g4 = 0; g4 < GP; g4 += 4) {
+          if (GP >= 4) {
+            const float4 x = *reinterpret_cast<const float4*>(prow + j * GP + g4);
+            pr[g4] = x.x; pr[g4 + 1] = x.y; pr[g4 + 2] = x.z; pr[g4 + 3] = x.w;
+          }
+        }
+        if (GP < 4) {
+#pragma unroll
+          for (int g = 0; g < GP; ++g) pr[g] = prow[j * GP + g];
+        }
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          acc[g][0] = fmaf(pr[g], v0, acc[g][0]);
+          acc[g][1] = fmaf(pr[g], v1, acc[g][1]);
+        }
+      }
+    }
+    if (!okv) aborted = true;
+  };
 
   for (int t = 0; t < T; ++t) {
     const int st = t % NK;
     const int kb = t1 - 1 - t;
     const bool okk = mbar_wait_warp(&k_full[st], (t / NK) & 1, fs);
-    // s_g = q_g . k_j for my key j
-    float s[kDecMaxG];
+    // ---- s_h = q_h . k_j for my key and my heads
+    float s[HPG];
 #pragma unroll
-    for (int g = 0; g < kDecMaxG; ++g) s[g] = 0.f;
-    const int key = kb * BK + tid;
-    if (okk && tid < BK) {
+    for (int h = 0; h < HPG; ++h) s[h] = 0.f;
+    if (okk && hbase < GP) {
       const uint32_t rowbase = sKa + st * TB;
 #pragma unroll 4
       for (int ch = 0; ch < D / 8; ++ch) {
         uint32_t a0, a1, a2, a3;
-        ld_shared_v4(rowbase + (ch >> 3) * (BK * 128) + sw128_offset(tid, ch & 7), a0, a1, a2, a3);
+        ld_shared_v4(rowbase + (ch >> 3) * (BK * 128) + sw128_offset(kj, ch & 7), a0, a1, a2, a3);
         const float kf[8] = {bf16lo_to_f32(a0), bf16hi_to_f32(a0), bf16lo_to_f32(a1), bf16hi_to_f32(a1),
                              bf16lo_to_f32(a2), bf16hi_to_f32(a2), bf16lo_to_f32(a3), bf16hi_to_f32(a3)};
 #pragma unroll
-        for (int g = 0; g < kDecMaxG; ++g) {
-          if (g < G) {
-            const float4 qa = *reinterpret_cast<const float4*>(sq + g * D + ch * 8);
-            const float4 qb = *reinterpret_cast<const float4*>(sq + g * D + ch * 8 + 4);
-            s[g] = fmaf(kf[0], qa.x, s[g]); s[g] = fmaf(kf[1], qa.y, s[g]);
-            s[g] = fmaf(kf[2], qa.z, s[g]); s[g] = fmaf(kf[3], qa.w, s[g]);
-            s[g] = fmaf(kf[4], qb.x, s[g]); s[g] = fmaf(kf[5], qb.y, s[g]);
-            s[g] = fmaf(kf[6], qb.z, s[g]); s[g] = fmaf(kf[7], qb.w, s[g]);
-          }
+        for (int h = 0; h < HPG; ++h) {
+          if (hbase + h >= GP) break;
+          const float* qr = sq + (hbase + h) * D + ch * 8;
+          const float4 qa = *reinterpret_cast<const float4*>(qr);
+          const float4 qb = *reinterpret_cast<const float4*>(qr + 4);
+          float a = s[h];
+          a = fmaf(kf[0], qa.x, a); a = fmaf(kf[1], qa.y, a); a = fmaf(kf[2], qa.z, a); a = fmaf(kf[3], qa.w, a);
+          a = fmaf(kf[4], qb.x, a); a = fmaf(kf[5], qb.y, a); a = fmaf(kf[6], qb.z, a); a = fmaf(kf[7], qb.w, a);
+          s[h] = a;
         }
       }
     }
-    mbar_arrive(&k_empty[st]);  // my key row has been read
-    const bool live = tid < BK && key < p.Lk;
+    mbar_arrive(&k_empty[st]);  // my reads of this K stage are done
+    const bool live = kb * BK + kj < p.Lk;
 #pragma unroll
-    for (int g = 0; g < kDecMaxG; ++g) {
-      float m = live ? s[g] : -INFINITY;
+    for (int h = 0; h < HPG; ++h) {
+      float m = live ? s[h] : -INFINITY;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (lane == 0 && g < G) sred[warp * kDecMaxG + g] = m;
+      if (lane == 0 && hbase + h < GP) sRmax[warp * GP + hbase + h] = m;
     }
     if (!okk) raise_abort(fs);
-    named_bar_sync(1, 128);
-    // ---- gates, one thread per head
+    named_bar_sync(1, NT);
+    // ---- gate, one thread per head (also folds in the previous kept tile's sums)
     if (tid < G) {
       const int g = tid;
-      float M = sred[g];
-      for (int w = 1; w < 4; ++w) M = fmaxf(M, sred[w * kDecMaxG + g]);
-      const float mu = smuse[g], l = sl[g];
+      const int w0 = (g / HPG) * WPG;  // the warps that scored head g
+      float M = sRmax[w0 * GP + g], sum = sRsum[w0 * GP + g];
+      for (int w = 1; w < WPG; ++w) {
+        M = fmaxf(M, sRmax[(w0 + w) * GP + g]);
+        sum += sRsum[(w0 + w) * GP + g];
+      }
+      float l = sL[g] + sum, mu = sM[g];
       const bool keep = (t == 0) || !kGate || (M * c2 >= mu + lg2_approx(l) + p.thr);
       float alpha = 1.f;
       if (keep) {
         const float mnew = fmaxf(mu, M * c2);
-        if (mnew > mu + 8.f) {
+        if (mnew > mu + 8.f) {  // lazy rescale: move the offset only when the max grew by > 2^8
           alpha = ex2_approx(mu - mnew);
-          sl[g] = l * alpha;
-          smuse[g] = mnew;
+          l *= alpha;
+          mu = mnew;
         }
       }
-      skeep[g] = keep ? 1.f : 0.f;
-      salpha[g] = alpha;
+      sL[g] = l;
+      sM[g] = mu;
+      sKeep[g] = keep ? 1.f : 0.f;
+      sAlpha[(nkept % NP) * GP + g] = alpha;
       my_cnt += keep ? 1 : 0;
       if (p.keep_map) p.keep_map[(static_cast<size_t>(b) * p.Hq + hq0 + g) * p.nk + kb] = keep ? 1 : 0;
     }
-    named_bar_sync(1, 128);
+    if (tid >= G && tid < GP) sAlpha[(nkept % NP) * GP + tid] = 1.f;
+    named_bar_sync(1, NT);
     if (tid == 0) {
       uint32_t any = 0;
-      for (int g = 0; g < G; ++g) any |= skeep[g] != 0.f ? 1u : 0u;
+      for (int g = 0; g < G; ++g) any |= sKeep[g] != 0.f ? 1u : 0u;
       if (abort_raised(fs)) any |= 2u;
-      if (any == 1u) {  // request V only now that a head keeps the tile
-        const int slot = nv % NV;
+      if (any == 1u) {  // V is requested only now that a head keeps the tile
+        const int vs = nkept % NV;
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&v_full[slot], TB);
+        mbar_arrive_expect_tx(&v_full[vs], TB);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(&tm_v, &v_full[slot], sV + slot * TB + h * (BK * 128), h * 64, hkv, kb * BK, b);
+          tma_load_4d(&tm_v, &v_full[vs], sV + vs * TB + h * (BK * 128), h * 64, hkv, kb * BK, b);
       }
       *sflag = any;
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(1, NT);
     const uint32_t flag = *reinterpret_cast<volatile uint32_t*>(sflag);
-    if (flag & 2u) break;
-    if (!(flag & 1u)) continue;
-    // ---- P for kept heads, row sums
+    if (flag & 2u) { aborted = true; break; }
+    // ---- probabilities of this tile for kept heads, and their per-warp sums
+    if (flag & 1u) {
+      float* prow = sP + (nkept % NP) * BK * GP;
 #pragma unroll
-    for (int g = 0; g < kDecMaxG; ++g) {
-      if (g < G) {
-        const float pv = (live && skeep[g] != 0.f) ? ex2_approx(fmaf(s[g], c2, -smuse[g])) : 0.f;
-        if (tid < BK) sp[g * BK + tid] = pv;
+      for (int h = 0; h < HPG; ++h) {
+        const int g = hbase + h;
+        float pv = 0.f;
+        if (g < GP && live && sKeep[g] != 0.f) pv = ex2_approx(fmaf(s[h], c2, -sM[g]));
+        if (g < GP) prow[kj * GP + g] = pv;
         float sum = pv;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0) sred[warp * kDecMaxG + g] = sum;
+        if (lane == 0 && g < GP) sRsum[warp * GP + g] = sum;
       }
+      ++nkept;
+    } else {
+#pragma unroll
+      for (int h = 0; h < HPG; ++h)
+        if (lane == 0 && hbase + h < GP) sRsum[warp * GP + hbase + h] = 0.f;
     }
-    const int slot = nv % NV;
-    const bool okv = mbar_wait_warp(&v_full[slot], (nv / NV) & 1, fs);
-    ++nv;
-    named_bar_sync(1, 128);
-    if (tid < G) sl[tid] += sred[tid] + sred[kDecMaxG + tid] + sred[2 * kDecMaxG + tid] + sred[3 * kDecMaxG + tid];
-    // ---- PV: thread tid owns output column tid of every head
-    if (okv && tid < D) {
-      float a[kDecMaxG];
-#pragma unroll
-      for (int g = 0; g < kDecMaxG; ++g) a[g] = g < G ? acc[g] * salpha[g] : 0.f;
-      const uint32_t vb = sVa + slot * TB + (tid >> 6) * (BK * 128) + ((tid & 7) << 1);
-      const uint32_t chunk = (tid & 63) >> 3;
-#pragma unroll 4
-      for (int j = 0; j < BK; ++j) {
-        const uint32_t addr = vb + j * 128 + ((chunk ^ (j & 7)) << 4);
-        unsigned short h;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(addr));
-        const float vv = __uint_as_float(static_cast<uint32_t>(h) << 16);
-#pragma unroll
-        for (int g = 0; g < kDecMaxG; ++g)
-          if (g < G) a[g] = fmaf(sp[g * BK + j], vv, a[g]);
-      }
-#pragma unroll
-      for (int g = 0; g < kDecMaxG; ++g) acc[g] = a[g];
-    }
-    named_bar_sync(1, 128);  // P, V slot and head state are reused by the next kept tile
+    // ---- PV of the kept tile kDecLag kept tiles back
+    if (nkept - ndone > kDecLag) run_pv(ndone++);  // its P was written at least one barrier ago
   }
 
-  // ---- partial results of this split
-  named_bar_sync(1, 128);
-  if (!abort_raised(fs)) {
-    if (tid < D) {
+  // ---- drain the pending PVs, then sum the key quarters
+  named_bar_sync(1, NT);
+  if (!aborted) {
+    while (ndone < nkept) run_pv(ndone++);
+  }
+  if (tid < G) {  // fold the last kept tile's sums into the normaliser
+    const int g = tid;
+    const int w0 = (g / HPG) * WPG;
+    float sum = 0.f;
+    for (int w = 0; w < WPG; ++w) sum += sRsum[(w0 + w) * GP + g];
+    sL[g] += sum;
+  }
+  named_bar_sync(1, NT);  // all PV reads of the rings are done; the K ring becomes the reduction buffer
+  float* ored = reinterpret_cast<float*>(sK);  // [4 quarters][GP][D]
+  if (2 * cp < D) {
 #pragma unroll
-      for (int g = 0; g < kDecMaxG; ++g)
-        if (g < G) {
-          const float l = sl[g];
-          p.o_part[((static_cast<size_t>(b) * p.Hq + hq0 + g) * p.n_splits + sp_idx) * D + tid] =
-              l > 0.f ? acc[g] / l : 0.f;
-        }
+    for (int g = 0; g < GP; ++g) {
+      ored[(kq * GP + g) * D + 2 * cp] = acc[g][0];
+      ored[(kq * GP + g) * D + 2 * cp + 1] = acc[g][1];
+    }
+  }
+  named_bar_sync(1, NT);
+  if (!aborted && !abort_raised(fs)) {
+    for (int i = tid; i < G * D; i += NT) {
+      const int g = i / D, c = i % D;
+      const float o = ored[(0 * GP + g) * D + c] + ored[(1 * GP + g) * D + c] + ored[(2 * GP + g) * D + c] +
+                      ored[(3 * GP + g) * D + c];
+      const float l = sL[g];
+      p.o_part[((static_cast<size_t>(b) * p.Hq + hq0 + g) * p.n_splits + sp_idx) * D + c] = l > 0.f ? o / l : 0.f;
     }
     if (tid < G) {
-      const float l = sl[tid];
+      const float l = sL[tid];
       p.lse_part[(static_cast<size_t>(b) * p.Hq + hq0 + tid) * p.n_splits + sp_idx] =
-          l > 0.f ? (smuse[tid] + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+          l > 0.f ? (sM[tid] + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
       atomicAdd(&p.kept_tiles[b * p.Hq + hq0 + tid], my_cnt);
     }
   }
   if (tid == 0)
-    for (int i = max(0, nv - NV); i < nv; ++i) mbar_wait_drain(&v_full[i % NV], (i / NV) & 1);
+    for (int i = max(0, nkept - NV); i < nkept; ++i) mbar_wait_drain(&v_full[i % NV], (i / NV) & 1);
 }
 
 // One warp per (b, query head): merge the split partials by their LSEs.
