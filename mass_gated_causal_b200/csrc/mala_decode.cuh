@@ -13,9 +13,11 @@
 // mala_decode_split_kernel: one CTA per (b, KV head, split). The split's key
 // tiles run newest -> oldest with a fresh online-softmax state per query
 // head; the newest tile of the split is always kept.
-//   warps 0-7  compute: for QK, thread t scores key t % BK against half of the
-//              GQA group's query heads; thread t < G also runs head t's gate
-//   warp  8    TMA producer of K tiles through an NK-stage ring
+//   warps 0-7  compute: for QK, thread t scores key t % BK against a share of
+//              the GQA group's query heads; P; PV
+//   warp  8    gate warp: lane g runs head g's gate for tile t (and requests
+//              V) while the compute warps score tile t + 1
+//   warp  9    TMA producer of K tiles through an NK-stage ring
 // The gate chain (QK, max, gate, normaliser update) never waits for V: the
 // state (m, l) follows from the scores alone. A kept tile's V TMA is issued
 // at its gate, its probabilities and rescale factors go to a ring, and its PV
@@ -58,8 +60,8 @@ struct DecLayout {
   static constexpr int OFF_Q = OFF_V + NV * T_BYTES;        // fp32 [GP][D]
   static constexpr int OFF_P = OFF_Q + GP * D * 4;            // fp32 [NP][BK][GP]
   static constexpr int OFF_ALPHA = OFF_P + NP * BK * GP * 4;  // fp32 [NP][GP]
-  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [8 warps][GP]
-  static constexpr int OFF_RSUM = OFF_RMAX + 8 * GP * 4;      // fp32 [8 warps][GP]
+  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [2 tiles][8 warps][GP]
+  static constexpr int OFF_RSUM = OFF_RMAX + 2 * 8 * GP * 4;  // fp32 [8 warps][GP]
   static constexpr int OFF_HEAD = OFF_RSUM + 8 * GP * 4;      // keep, m, l per head
   static constexpr int OFF_BAR = OFF_HEAD + 3 * GP * 4;
   static constexpr int N_BARS = 2 * NK + NV;                  // k_full, k_empty, v_full
@@ -72,7 +74,7 @@ struct DecLayout {
 };
 
 template <int D, int BK, int GP, bool kGate>
-__global__ void __launch_bounds__(288, 1)
+__global__ void __launch_bounds__(320, 1)
     mala_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                              const DecParams p) {
   using Lay = DecLayout<D, BK, GP>;
@@ -81,7 +83,9 @@ __global__ void __launch_bounds__(288, 1)
   constexpr int HPG = (GP + NGRP - 1) / NGRP;    // query heads scored per thread
   constexpr int WPG = BK / 32;                   // warps per group
   constexpr int KQ = BK / 4;                     // keys per PV quarter
+  constexpr int NB = NT + 32;                    // threads in the per-tile barriers (compute + gate warp)
   static_assert(D == 128 || D == 64, "head dim");
+  static_assert(KQ % 8 == 0, "PV unrolls by the 8-row swizzle period");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + Lay::OFF_K;
@@ -89,8 +93,8 @@ __global__ void __launch_bounds__(288, 1)
   float* sq = reinterpret_cast<float*>(smem + Lay::OFF_Q);
   float* sP = reinterpret_cast<float*>(smem + Lay::OFF_P);
   float* sAlpha = reinterpret_cast<float*>(smem + Lay::OFF_ALPHA);
-  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);
-  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);
+  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);  // [2 tiles][8 warps][GP]
+  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);  // [8 warps][GP]
   float* sKeep = reinterpret_cast<float*>(smem + Lay::OFF_HEAD);
   float* sM = sKeep + GP;  // exponent offset per head (log2 units)
   float* sL = sM + GP;     // running normaliser per head
@@ -143,7 +147,7 @@ __global__ void __launch_bounds__(288, 1)
   for (int i = tid; i < 8 * GP; i += blockDim.x) sRsum[i] = 0.f;
   __syncthreads();
 
-  if (warp == 8) {
+  if (warp == 9) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
@@ -158,75 +162,110 @@ __global__ void __launch_bounds__(288, 1)
       for (int t = max(0, issued - NK); t < issued; ++t) mbar_wait_drain(&k_full[t % NK], (t / NK) & 1);
     }
     __syncwarp();
-    return;  // the compute warps below synchronise with named barrier 1 only
+    return;  // the other warps synchronise with named barriers 1 (compute + gate) and 2 (compute)
+  }
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ gate warp
+    // Lane g < G gates head g for tile t while the compute warps score tile t+1.
+    int my_cnt = 0, nkept = 0;
+    bool aborted = false;
+    for (int t = 0; t < T; ++t) {
+      const int kb = t1 - 1 - t;
+      named_bar_sync(1, NB);  // A: maxima of tile t and sums of the previous kept tile are in place
+      bool keep = false;
+      if (lane < G) {
+        const int g = lane;
+        const int w0 = (g / HPG) * WPG;  // the warps that scored head g
+        const float* rm = sRmax + (t & 1) * 8 * GP;
+        float M = rm[w0 * GP + g], sum = sRsum[w0 * GP + g];
+        for (int w = 1; w < WPG; ++w) {
+          M = fmaxf(M, rm[(w0 + w) * GP + g]);
+          sum += sRsum[(w0 + w) * GP + g];
+        }
+        float l = sL[g] + sum, mu = sM[g];
+        keep = (t == 0) || !kGate || (M * p.scale_log2 >= mu + lg2_approx(l) + p.thr);
+        float alpha = 1.f;
+        if (keep) {
+          const float mnew = fmaxf(mu, M * p.scale_log2);
+          if (mnew > mu + 8.f) {  // lazy rescale: move the offset only when the max grew by > 2^8
+            alpha = ex2_approx(mu - mnew);
+            l *= alpha;
+            mu = mnew;
+          }
+        }
+        sL[g] = l;
+        sM[g] = mu;
+        sKeep[g] = keep ? 1.f : 0.f;
+        sAlpha[(nkept % NP) * GP + g] = alpha;
+        my_cnt += keep ? 1 : 0;
+        if (p.keep_map) p.keep_map[(static_cast<size_t>(b) * p.Hq + hq0 + g) * p.nk + kb] = keep ? 1 : 0;
+      } else if (lane < GP) {
+        sAlpha[(nkept % NP) * GP + lane] = 1.f;
+      }
+      const bool any = __ballot_sync(0xffffffffu, keep) != 0u;
+      if (lane == 0) {
+        const bool ab = abort_raised(fs);
+        if (any && !ab) {  // V is requested only now that a head keeps the tile
+          const int vs = nkept % NV;
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&v_full[vs], TB);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(&tm_v, &v_full[vs], sV + vs * TB + h * (BK * 128), h * 64, hkv, kb * BK, b);
+        }
+        *sflag = (any ? 1u : 0u) | (ab ? 2u : 0u);
+        aborted = ab;
+      }
+      aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
+      if (any) ++nkept;
+      named_bar_sync(1, NB);  // B: the decision of tile t is visible
+      if (aborted) break;
+    }
+    named_bar_sync(1, NB);  // C: the last probabilities and sums are written
+    if (!aborted && lane < G) {
+      const int g = lane;
+      const int w0 = (g / HPG) * WPG;
+      float sum = 0.f;
+      for (int w = 0; w < WPG; ++w) sum += sRsum[(w0 + w) * GP + g];
+      sL[g] += sum;  // fold the last kept tile into the normaliser
+    }
+    named_bar_sync(1, NB);  // D: the compute warps have summed the key quarters
+    if (!aborted && !abort_raised(fs) && lane < G) {
+      const float l = sL[lane];
+      p.lse_part[(static_cast<size_t>(b) * p.Hq + hq0 + lane) * p.n_splits + sp_idx] =
+          l > 0.f ? (sM[lane] + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+      atomicAdd(&p.kept_tiles[b * p.Hq + hq0 + lane], my_cnt);
+    }
+    if (lane == 0)
+      for (int i = max(0, nkept - NV); i < nkept; ++i) mbar_wait_drain(&v_full[i % NV], (i / NV) & 1);
+    return;
   }
 
   // ---------------------------------------------------------- compute warps
   const float c2 = p.scale_log2;
-  const int kj = tid % BK;        // QK: my key within the tile
+  const int kj = tid % BK;             // QK: my key within the tile
   const int hbase = (tid / BK) * HPG;  // QK: first of my heads
-  const int cp = tid & 63;        // PV: my output column pair (D = 128) / column (D = 64, cp < 32 pairs)
-  const int kq = tid >> 6;        // PV: my quarter of the keys
+  const int cp = tid & 63;             // PV: my output column pair
+  const int kq = tid >> 6;             // PV: my quarter of the keys
   float acc[GP][2];
 #pragma unroll
   for (int g = 0; g < GP; ++g) acc[g][0] = acc[g][1] = 0.f;
-  int my_cnt = 0;   // tiles kept by head tid (threads tid < G)
-  int nkept = 0;    // kept tiles so far (V loads issued)
-  int ndone = 0;    // kept tiles whose PV has run
+  int nkept = 0;  // kept tiles so far
+  int ndone = 0;  // kept tiles whose PV has run
   const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
   bool aborted = false;
 
-  auto run_pv = [&](int n) {  // PV of the n-th kept tile (all compute threads)
-    const int vs = n % NV, ps = n % NP;
-    const bool okv = mbar_wait_warp(&v_full[vs], (n / NV) & 1, fs);
-    if (okv && 2 * cp < D) {
-      float al[GP];
-#pragma unroll
-      for (int g = 0; g < GP; ++g) al[g] = sAlpha[ps * GP + g];
-#pragma unroll
-      for (int g = 0; g < GP; ++g) { acc[g][0] *= al[g]; acc[g][1] *= al[g]; }
-      const int col = 2 * cp;
-      const uint32_t vb = sVa + vs * TB + (col >> 6) * (BK * 128) + ((col & 7) << 1);
-      const uint32_t chunk = (col & 63) >> 3;
-      const float* prow = sP + ps * BK * GP;
-#pragma unroll 4
-      for (int jj = 0; jj < KQ; ++jj) {
-        const int j = kq * KQ + jj;
-        uint32_t v2;
-        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v2) : "r"(vb + j * 128 + ((chunk ^ (j & 7)) << 4)));
-        const float v0 = bf16lo_to_f32(v2), v1 = bf16hi_to_f32(v2);
-        float pr[GP];
-#pragma unroll
-        for (int g4 = 0; g4 < GP; g4 += 4) {
-          if (GP >= 4) {
-            const float4 x = *reinterpret_cast<const float4*>(prow + j * GP + g4);
-            pr[g4] = x.x; pr[g4 + 1] = x.y; pr[g4 + 2] = x.z; pr[g4 + 3] = x.w;
-          }
-        }
-        if (GP < 4) {
-#pragma unroll
-          for (int g = 0; g < GP; ++g) pr[g] = prow[j * GP + g];
-        }
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          acc[g][0] = fmaf(pr[g], v0, acc[g][0]);
-          acc[g][1] = fmaf(pr[g], v1, acc[g][1]);
-        }
-      }
-    }
-    if (!okv) aborted = true;
-  };
-
-  for (int t = 0; t < T; ++t) {
+  auto score = [&](int t, float (&s)[HPG]) {  // s_h = q_h . k_j for my key of tile t and my heads
     const int st = t % NK;
     const int kb = t1 - 1 - t;
     const bool okk = mbar_wait_warp(&k_full[st], (t / NK) & 1, fs);
-    // ---- s_h = q_h . k_j for my key and my heads
-    float s[HPG];
 #pragma unroll
     for (int h = 0; h < HPG; ++h) s[h] = 0.f;
     if (okk && hbase < GP) {
       const uint32_t rowbase = sKa + st * TB;
+      float part[HPG][4];  // four independent partial sums per head (instruction-level parallelism)
+#pragma unroll
+      for (int h = 0; h < HPG; ++h) part[h][0] = part[h][1] = part[h][2] = part[h][3] = 0.f;
 #pragma unroll 4
       for (int ch = 0; ch < D / 8; ++ch) {
         uint32_t a0, a1, a2, a3;
@@ -239,12 +278,14 @@ __global__ void __launch_bounds__(288, 1)
           const float* qr = sq + (hbase + h) * D + ch * 8;
           const float4 qa = *reinterpret_cast<const float4*>(qr);
           const float4 qb = *reinterpret_cast<const float4*>(qr + 4);
-          float a = s[h];
-          a = fmaf(kf[0], qa.x, a); a = fmaf(kf[1], qa.y, a); a = fmaf(kf[2], qa.z, a); a = fmaf(kf[3], qa.w, a);
-          a = fmaf(kf[4], qb.x, a); a = fmaf(kf[5], qb.y, a); a = fmaf(kf[6], qb.z, a); a = fmaf(kf[7], qb.w, a);
-          s[h] = a;
+          part[h][0] = fmaf(kf[0], qa.x, part[h][0]); part[h][1] = fmaf(kf[1], qa.y, part[h][1]);
+          part[h][2] = fmaf(kf[2], qa.z, part[h][2]); part[h][3] = fmaf(kf[3], qa.w, part[h][3]);
+          part[h][0] = fmaf(kf[4], qb.x, part[h][0]); part[h][1] = fmaf(kf[5], qb.y, part[h][1]);
+          part[h][2] = fmaf(kf[6], qb.z, part[h][2]); part[h][3] = fmaf(kf[7], qb.w, part[h][3]);
         }
       }
+#pragma unroll
+      for (int h = 0; h < HPG; ++h) s[h] = (part[h][0] + part[h][1]) + (part[h][2] + part[h][3]);
     }
     mbar_arrive(&k_empty[st]);  // my reads of this K stage are done
     const bool live = kb * BK + kj < p.Lk;
@@ -253,63 +294,72 @@ __global__ void __launch_bounds__(288, 1)
       float m = live ? s[h] : -INFINITY;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (lane == 0 && hbase + h < GP) sRmax[warp * GP + hbase + h] = m;
+      if (lane == 0 && hbase + h < GP) sRmax[((t & 1) * 8 + warp) * GP + hbase + h] = m;
     }
     if (!okk) raise_abort(fs);
-    named_bar_sync(1, NT);
-    // ---- gate, one thread per head (also folds in the previous kept tile's sums)
-    if (tid < G) {
-      const int g = tid;
-      const int w0 = (g / HPG) * WPG;  // the warps that scored head g
-      float M = sRmax[w0 * GP + g], sum = sRsum[w0 * GP + g];
-      for (int w = 1; w < WPG; ++w) {
-        M = fmaxf(M, sRmax[(w0 + w) * GP + g]);
-        sum += sRsum[(w0 + w) * GP + g];
+  };
+
+  auto run_pv = [&](int n) {  // PV of the n-th kept tile (all compute threads)
+    const int vs = n % NV, ps = n % NP;
+    const bool okv = mbar_wait_warp(&v_full[vs], (n / NV) & 1, fs);
+    if (okv && 2 * cp < D) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float al = sAlpha[ps * GP + g];
+        acc[g][0] *= al;
+        acc[g][1] *= al;
       }
-      float l = sL[g] + sum, mu = sM[g];
-      const bool keep = (t == 0) || !kGate || (M * c2 >= mu + lg2_approx(l) + p.thr);
-      float alpha = 1.f;
-      if (keep) {
-        const float mnew = fmaxf(mu, M * c2);
-        if (mnew > mu + 8.f) {  // lazy rescale: move the offset only when the max grew by > 2^8
-          alpha = ex2_approx(mu - mnew);
-          l *= alpha;
-          mu = mnew;
+      const int col = 2 * cp;
+      const uint32_t chunk = (col & 63) >> 3;
+      const uint32_t vb = sVa + vs * TB + (col >> 6) * (BK * 128) + ((col & 7) << 1) + kq * KQ * 128;
+      const float* prow = sP + (ps * BK + kq * KQ) * GP;
+#pragma unroll 1
+      for (int m8 = 0; m8 < KQ / 8; ++m8) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {  // row j = kq*KQ + 8*m8 + r has j % 8 == r
+          const int jl = m8 * 8 + r;
+          uint32_t v2;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v2) : "r"(vb + jl * 128 + ((chunk ^ r) << 4)));
+          const float v0 = bf16lo_to_f32(v2), v1 = bf16hi_to_f32(v2);
+          float pr[GP];
+          if (GP >= 4) {
+#pragma unroll
+            for (int g4 = 0; g4 < GP; g4 += 4) {
+              const float4 x = *reinterpret_cast<const float4*>(prow + jl * GP + g4);
+              pr[g4] = x.x; pr[g4 + 1] = x.y; pr[g4 + 2] = x.z; pr[g4 + 3] = x.w;
+            }
+          } else {
+#pragma unroll
+            for (int g = 0; g < GP; ++g) pr[g] = prow[jl * GP + g];
+          }
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            acc[g][0] = fmaf(pr[g], v0, acc[g][0]);
+            acc[g][1] = fmaf(pr[g], v1, acc[g][1]);
+          }
         }
       }
-      sL[g] = l;
-      sM[g] = mu;
-      sKeep[g] = keep ? 1.f : 0.f;
-      sAlpha[(nkept % NP) * GP + g] = alpha;
-      my_cnt += keep ? 1 : 0;
-      if (p.keep_map) p.keep_map[(static_cast<size_t>(b) * p.Hq + hq0 + g) * p.nk + kb] = keep ? 1 : 0;
     }
-    if (tid >= G && tid < GP) sAlpha[(nkept % NP) * GP + tid] = 1.f;
-    named_bar_sync(1, NT);
-    if (tid == 0) {
-      uint32_t any = 0;
-      for (int g = 0; g < G; ++g) any |= sKeep[g] != 0.f ? 1u : 0u;
-      if (abort_raised(fs)) any |= 2u;
-      if (any == 1u) {  // V is requested only now that a head keeps the tile
-        const int vs = nkept % NV;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&v_full[vs], TB);
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(&tm_v, &v_full[vs], sV + vs * TB + h * (BK * 128), h * 64, hkv, kb * BK, b);
-      }
-      *sflag = any;
-    }
-    named_bar_sync(1, NT);
+    if (!okv) aborted = true;
+  };
+
+  float s_cur[HPG], s_nxt[HPG];
+  score(0, s_cur);
+  for (int t = 0; t < T; ++t) {
+    const int kb = t1 - 1 - t;
+    named_bar_sync(1, NB);            // A: maxima of tile t are in place
+    if (t + 1 < T) score(t + 1, s_nxt);  // overlaps the gate of tile t
+    named_bar_sync(1, NB);            // B: the decision of tile t is visible
     const uint32_t flag = *reinterpret_cast<volatile uint32_t*>(sflag);
     if (flag & 2u) { aborted = true; break; }
-    // ---- probabilities of this tile for kept heads, and their per-warp sums
-    if (flag & 1u) {
+    const bool live = kb * BK + kj < p.Lk;
+    if (flag & 1u) {  // probabilities of tile t for kept heads, and their per-warp sums
       float* prow = sP + (nkept % NP) * BK * GP;
 #pragma unroll
       for (int h = 0; h < HPG; ++h) {
         const int g = hbase + h;
         float pv = 0.f;
-        if (g < GP && live && sKeep[g] != 0.f) pv = ex2_approx(fmaf(s[h], c2, -sM[g]));
+        if (g < GP && live && sKeep[g] != 0.f) pv = ex2_approx(fmaf(s_cur[h], c2, -sM[g]));
         if (g < GP) prow[kj * GP + g] = pv;
         float sum = pv;
 #pragma unroll
@@ -322,24 +372,17 @@ __global__ void __launch_bounds__(288, 1)
       for (int h = 0; h < HPG; ++h)
         if (lane == 0 && hbase + h < GP) sRsum[warp * GP + hbase + h] = 0.f;
     }
-    // ---- PV of the kept tile kDecLag kept tiles back
     if (nkept - ndone > kDecLag) run_pv(ndone++);  // its P was written at least one barrier ago
+#pragma unroll
+    for (int h = 0; h < HPG; ++h) s_cur[h] = s_nxt[h];
   }
 
-  // ---- drain the pending PVs, then sum the key quarters
-  named_bar_sync(1, NT);
+  named_bar_sync(1, NB);  // C
   if (!aborted) {
     while (ndone < nkept) run_pv(ndone++);
   }
-  if (tid < G) {  // fold the last kept tile's sums into the normaliser
-    const int g = tid;
-    const int w0 = (g / HPG) * WPG;
-    float sum = 0.f;
-    for (int w = 0; w < WPG; ++w) sum += sRsum[(w0 + w) * GP + g];
-    sL[g] += sum;
-  }
-  named_bar_sync(1, NT);  // all PV reads of the rings are done; the K ring becomes the reduction buffer
-  float* ored = reinterpret_cast<float*>(sK);  // [4 quarters][GP][D]
+  named_bar_sync(2, NT);  // compute warps only (barrier 2): every PV read of the rings is done
+  float* ored = reinterpret_cast<float*>(sK);  // [4 quarters][GP][D], reuses the K ring
   if (2 * cp < D) {
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -347,7 +390,7 @@ __global__ void __launch_bounds__(288, 1)
       ored[(kq * GP + g) * D + 2 * cp + 1] = acc[g][1];
     }
   }
-  named_bar_sync(1, NT);
+  named_bar_sync(1, NB);  // D (with the gate warp, which has folded the last sums into sL)
   if (!aborted && !abort_raised(fs)) {
     for (int i = tid; i < G * D; i += NT) {
       const int g = i / D, c = i % D;
@@ -356,15 +399,7 @@ __global__ void __launch_bounds__(288, 1)
       const float l = sL[g];
       p.o_part[((static_cast<size_t>(b) * p.Hq + hq0 + g) * p.n_splits + sp_idx) * D + c] = l > 0.f ? o / l : 0.f;
     }
-    if (tid < G) {
-      const float l = sL[tid];
-      p.lse_part[(static_cast<size_t>(b) * p.Hq + hq0 + tid) * p.n_splits + sp_idx] =
-          l > 0.f ? (sM[tid] + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
-      atomicAdd(&p.kept_tiles[b * p.Hq + hq0 + tid], my_cnt);
-    }
   }
-  if (tid == 0)
-    for (int i = max(0, nkept - NV); i < nkept; ++i) mbar_wait_drain(&v_full[i % NV], (i / NV) & 1);
 }
 
 // One warp per (b, query head): merge the split partials by their LSEs.
