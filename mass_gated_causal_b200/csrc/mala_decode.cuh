@@ -13,16 +13,16 @@
 // mala_decode_split_kernel: one CTA per (b, KV head, split). The split's key
 // tiles run newest -> oldest with a fresh online-softmax state per query
 // head; the newest tile of the split is always kept.
-//   warps 0-7  compute: for QK, thread t scores key t % BK against a share of
+//   warps 0-15 compute: for QK, thread t scores key t % BK against a share of
 //              the GQA group's query heads; P; PV
-//   warp  8    gate warp: lane g runs head g's gate for tile t (and requests
+//   warp  16   gate warp: lane g runs head g's gate for tile t (and requests
 //              V) while the compute warps score tile t + 1
-//   warp  9    TMA producer of K tiles through an NK-stage ring
+//   warp  17   TMA producer of K tiles through an NK-stage ring
 // The gate chain (QK, max, gate, normaliser update) never waits for V: the
 // state (m, l) follows from the scores alone. A kept tile's V TMA is issued
 // at its gate, its probabilities and rescale factors go to a ring, and its PV
 // runs kLag kept tiles later, when V has had time to land. PV maps thread t to
-// an output column pair and a quarter of the keys; the quarters are summed at
+// an output column pair and a quarter of the keys; the slices are summed at
 // the end of the split. Each split writes (O_s, LSE_s) per head.
 //
 // mala_decode_combine_kernel: LSE = log sum_s exp(LSE_s),
@@ -53,28 +53,28 @@ struct DecLayout {
   static constexpr int NK = 3;
   static constexpr int NV = kDecLag + 1;
   static constexpr int NP = kDecLag + 1;
-  static constexpr int NT = 256;  // compute threads
+  static constexpr int NT = 512;  // compute threads
   static constexpr int T_BYTES = BK * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * T_BYTES;
   static constexpr int OFF_Q = OFF_V + NV * T_BYTES;        // fp32 [GP][D]
   static constexpr int OFF_P = OFF_Q + GP * D * 4;            // fp32 [NP][BK][GP]
   static constexpr int OFF_ALPHA = OFF_P + NP * BK * GP * 4;  // fp32 [NP][GP]
-  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [2 tiles][8 warps][GP]
-  static constexpr int OFF_RSUM = OFF_RMAX + 2 * 8 * GP * 4;  // fp32 [8 warps][GP]
-  static constexpr int OFF_HEAD = OFF_RSUM + 8 * GP * 4;      // keep, m, l per head
+  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [2 tiles][16 warps][GP]
+  static constexpr int OFF_RSUM = OFF_RMAX + 2 * 16 * GP * 4; // fp32 [16 warps][GP]
+  static constexpr int OFF_HEAD = OFF_RSUM + 16 * GP * 4;     // keep, m, l per head
   static constexpr int OFF_BAR = OFF_HEAD + 3 * GP * 4;
   static constexpr int N_BARS = 2 * NK + NV;                  // k_full, k_empty, v_full
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
-  static constexpr int ORED_BYTES = 4 * GP * D * 4;           // end-of-split reduction, reuses the K ring
+  static constexpr int ORED_BYTES = 8 * GP * D * 4;           // end-of-split reduction, reuses the K ring
   static_assert(ORED_BYTES <= NK * T_BYTES, "reduction buffer must fit in the K ring");
   static_assert(ALLOC_BYTES <= 232448, "decode shared memory exceeds the per-CTA limit");
 };
 
 template <int D, int BK, int GP, bool kGate>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     mala_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                              const DecParams p) {
   using Lay = DecLayout<D, BK, GP>;
@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int NGRP = NT / BK;                  // QK thread groups (one key per thread per group)
   constexpr int HPG = (GP + NGRP - 1) / NGRP;    // query heads scored per thread
   constexpr int WPG = BK / 32;                   // warps per group
-  constexpr int KQ = BK / 4;                     // keys per PV quarter
+  constexpr int NKQ = NT / 64;                   // PV key slices (64 column pairs each)
+  constexpr int KQ = BK / NKQ;                   // keys per PV slice
   constexpr int NB = NT + 32;                    // threads in the per-tile barriers (compute + gate warp)
   static_assert(D == 128 || D == 64, "head dim");
   static_assert(KQ % 8 == 0, "PV unrolls by the 8-row swizzle period");
@@ -93,8 +94,8 @@ __global__ void __launch_bounds__(320, 1)
   float* sq = reinterpret_cast<float*>(smem + Lay::OFF_Q);
   float* sP = reinterpret_cast<float*>(smem + Lay::OFF_P);
   float* sAlpha = reinterpret_cast<float*>(smem + Lay::OFF_ALPHA);
-  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);  // [2 tiles][8 warps][GP]
-  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);  // [8 warps][GP]
+  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);  // [2 tiles][16 warps][GP]
+  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);  // [16 warps][GP]
   float* sKeep = reinterpret_cast<float*>(smem + Lay::OFF_HEAD);
   float* sM = sKeep + GP;  // exponent offset per head (log2 units)
   float* sL = sM + GP;     // running normaliser per head
@@ -144,10 +145,10 @@ __global__ void __launch_bounds__(320, 1)
     sL[tid] = 0.f;
     sKeep[tid] = 0.f;  // padded heads (G < GP) never keep
   }
-  for (int i = tid; i < 8 * GP; i += blockDim.x) sRsum[i] = 0.f;
+  for (int i = tid; i < 16 * GP; i += blockDim.x) sRsum[i] = 0.f;
   __syncthreads();
 
-  if (warp == 9) {
+  if (warp == 17) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(320, 1)
     return;  // the other warps synchronise with named barriers 1 (compute + gate) and 2 (compute)
   }
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ gate warp
     // Lane g < G gates head g for tile t while the compute warps score tile t+1.
     int my_cnt = 0, nkept = 0;
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(320, 1)
       if (lane < G) {
         const int g = lane;
         const int w0 = (g / HPG) * WPG;  // the warps that scored head g
-        const float* rm = sRmax + (t & 1) * 8 * GP;
+        const float* rm = sRmax + (t & 1) * 16 * GP;
         float M = rm[w0 * GP + g], sum = sRsum[w0 * GP + g];
         for (int w = 1; w < WPG; ++w) {
           M = fmaxf(M, rm[(w0 + w) * GP + g]);
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(320, 1)
   const int kj = tid % BK;             // QK: my key within the tile
   const int hbase = (tid / BK) * HPG;  // QK: first of my heads
   const int cp = tid & 63;             // PV: my output column pair
-  const int kq = tid >> 6;             // PV: my quarter of the keys
+  const int kq = tid >> 6;             // PV: my slice of the keys
   float acc[GP][2];
 #pragma unroll
   for (int g = 0; g < GP; ++g) acc[g][0] = acc[g][1] = 0.f;
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(320, 1)
       float m = live ? s[h] : -INFINITY;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (lane == 0 && hbase + h < GP) sRmax[((t & 1) * 8 + warp) * GP + hbase + h] = m;
+      if (lane == 0 && hbase + h < GP) sRmax[((t & 1) * 16 + warp) * GP + hbase + h] = m;
     }
     if (!okk) raise_abort(fs);
   };
@@ -382,7 +383,7 @@ __global__ void __launch_bounds__(320, 1)
     while (ndone < nkept) run_pv(ndone++);
   }
   named_bar_sync(2, NT);  // compute warps only (barrier 2): every PV read of the rings is done
-  float* ored = reinterpret_cast<float*>(sK);  // [4 quarters][GP][D], reuses the K ring
+  float* ored = reinterpret_cast<float*>(sK);  // [NKQ slices][GP][D], reuses the K ring
   if (2 * cp < D) {
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -394,8 +395,9 @@ __global__ void __launch_bounds__(320, 1)
   if (!aborted && !abort_raised(fs)) {
     for (int i = tid; i < G * D; i += NT) {
       const int g = i / D, c = i % D;
-      const float o = ored[(0 * GP + g) * D + c] + ored[(1 * GP + g) * D + c] + ored[(2 * GP + g) * D + c] +
-                      ored[(3 * GP + g) * D + c];
+      float o = 0.f;
+#pragma unroll
+      for (int x = 0; x < NKQ; ++x) o += ored[(x * GP + g) * D + c];
       const float l = sL[g];
       p.o_part[((static_cast<size_t>(b) * p.Hq + hq0 + g) * p.n_splits + sp_idx) * D + c] = l > 0.f ? o / l : 0.f;
     }

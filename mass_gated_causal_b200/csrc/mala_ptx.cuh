@@ -59,6 +59,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended until the phase completes or the hint (ns) expires, instead of
+// spinning and taking issue slots from the warps doing the work.
+constexpr uint32_t kSuspendHintNs = 65536;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared per-CTA failure state used by the bounded waits.
 struct FailState {
   int* abort_flag;     // shared memory: set once any wait in the CTA gave up
@@ -80,8 +96,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 15u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((n & 3u) == 0) {
       if (abort_raised(fs)) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         raise_abort(fs);
@@ -97,9 +113,9 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, c
   if (__all_sync(0xffffffffu, ok)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
-    ok = mbar_try_wait(bar, parity);
+    ok = mbar_try_wait_sleep(bar, parity);
     if (__all_sync(0xffffffffu, ok)) return true;
-    if ((n & 15u) == 0) {
+    if ((n & 3u) == 0) {
       int give_up = 0;
       if ((threadIdx.x & 31) == 0) {
         give_up = abort_raised(fs) ? 1 : 0;
@@ -120,8 +136,8 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 15u) == 0 && global_timer_ns() - t0 > kDrainLimitNs) return false;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((n & 3u) == 0 && global_timer_ns() - t0 > kDrainLimitNs) return false;
   }
 }
 
