@@ -134,7 +134,7 @@ int launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecPara
   auto kern = mala::mala_decode_split_kernel<D, BK, GP, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hkv * p.n_splits;
-  kern<<<grid, 576, Lay::ALLOC_BYTES, st>>>(mk, mv, p);
+  kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 

@@ -53,49 +53,50 @@ struct DecLayout {
   static constexpr int NK = 3;
   static constexpr int NV = kDecLag + 1;
   static constexpr int NP = kDecLag + 1;
-  static constexpr int NT = 512;  // compute threads
+  static constexpr int NW = 8;          // compute warps
+  static constexpr int NT = NW * 32;    // compute threads
+  static constexpr int LPK = D / 8;     // lanes per key row (one 16-byte chunk each)
+  static constexpr int KPW = 32 / LPK;  // keys per warp step
+  static constexpr int NPART = NW;      // partial O accumulators (one per warp) summed at the end
   static constexpr int T_BYTES = BK * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + NK * T_BYTES;
   static constexpr int OFF_Q = OFF_V + NV * T_BYTES;        // fp32 [GP][D]
-  static constexpr int OFF_P = OFF_Q + GP * D * 4;            // fp32 [NP][BK][GP]
-  static constexpr int OFF_ALPHA = OFF_P + NP * BK * GP * 4;  // fp32 [NP][GP]
-  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [2 tiles][16 warps][GP]
-  static constexpr int OFF_RSUM = OFF_RMAX + 2 * 16 * GP * 4; // fp32 [16 warps][GP]
-  static constexpr int OFF_HEAD = OFF_RSUM + 16 * GP * 4;     // keep, m, l per head
+  static constexpr int OFF_ALPHA = OFF_Q + GP * D * 4;        // fp32 [NP][GP]
+  static constexpr int OFF_RMAX = OFF_ALPHA + NP * GP * 4;    // fp32 [2 tiles][NW][GP]
+  static constexpr int OFF_RSUM = OFF_RMAX + 2 * NW * GP * 4; // fp32 [NW][GP]
+  static constexpr int OFF_HEAD = OFF_RSUM + NW * GP * 4;     // keep, m, l per head
   static constexpr int OFF_BAR = OFF_HEAD + 3 * GP * 4;
   static constexpr int N_BARS = 2 * NK + NV;                  // k_full, k_empty, v_full
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
-  static constexpr int ORED_BYTES = 8 * GP * D * 4;           // end-of-split reduction, reuses the K ring
+  static constexpr int ORED_BYTES = NPART * GP * D * 4;       // end-of-split reduction, reuses the K ring
   static_assert(ORED_BYTES <= NK * T_BYTES, "reduction buffer must fit in the K ring");
   static_assert(ALLOC_BYTES <= 232448, "decode shared memory exceeds the per-CTA limit");
 };
 
 template <int D, int BK, int GP, bool kGate>
-__global__ void __launch_bounds__(576, 1)
+__global__ void __launch_bounds__(320, 1)
     mala_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                              const DecParams p) {
   using Lay = DecLayout<D, BK, GP>;
-  constexpr int NK = Lay::NK, NV = Lay::NV, NP = Lay::NP, TB = Lay::T_BYTES, NT = Lay::NT;
-  constexpr int NGRP = NT / BK;                  // QK thread groups (one key per thread per group)
-  constexpr int HPG = (GP + NGRP - 1) / NGRP;    // query heads scored per thread
-  constexpr int WPG = BK / 32;                   // warps per group
-  constexpr int NKQ = NT / 64;                   // PV key slices (64 column pairs each)
-  constexpr int KQ = BK / NKQ;                   // keys per PV slice
-  constexpr int NB = NT + 32;                    // threads in the per-tile barriers (compute + gate warp)
+  constexpr int NK = Lay::NK, NV = Lay::NV, NP = Lay::NP, TB = Lay::T_BYTES;
+  constexpr int NW = Lay::NW, NT = Lay::NT, LPK = Lay::LPK, KPW = Lay::KPW;
+  constexpr int KPWT = BK / NW;      // keys per warp per tile
+  constexpr int STEPS = KPWT / KPW;  // warp steps per tile
+  constexpr int NB = NT + 32;        // threads in the per-tile barriers (compute + gate warp)
   static_assert(D == 128 || D == 64, "head dim");
-  static_assert(KQ % 8 == 0, "PV unrolls by the 8-row swizzle period");
+  static_assert(STEPS >= 1 && KPWT % KPW == 0, "tile shape");
+  static_assert(GP <= LPK, "one lane per head within a key row");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + Lay::OFF_K;
   uint8_t* sV = smem + Lay::OFF_V;
   float* sq = reinterpret_cast<float*>(smem + Lay::OFF_Q);
-  float* sP = reinterpret_cast<float*>(smem + Lay::OFF_P);
   float* sAlpha = reinterpret_cast<float*>(smem + Lay::OFF_ALPHA);
-  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);  // [2 tiles][16 warps][GP]
-  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);  // [16 warps][GP]
+  float* sRmax = reinterpret_cast<float*>(smem + Lay::OFF_RMAX);
+  float* sRsum = reinterpret_cast<float*>(smem + Lay::OFF_RSUM);
   float* sKeep = reinterpret_cast<float*>(smem + Lay::OFF_HEAD);
   float* sM = sKeep + GP;  // exponent offset per head (log2 units)
   float* sL = sM + GP;     // running normaliser per head
@@ -145,10 +146,10 @@ __global__ void __launch_bounds__(576, 1)
     sL[tid] = 0.f;
     sKeep[tid] = 0.f;  // padded heads (G < GP) never keep
   }
-  for (int i = tid; i < 16 * GP; i += blockDim.x) sRsum[i] = 0.f;
+  for (int i = tid; i < NW * GP; i += blockDim.x) sRsum[i] = 0.f;
   __syncthreads();
 
-  if (warp == 17) {
+  if (warp == NW + 1) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(576, 1)
     return;  // the other warps synchronise with named barriers 1 (compute + gate) and 2 (compute)
   }
 
-  if (warp == 16) {
+  if (warp == NW) {
     // ------------------------------------------------------------ gate warp
     // Lane g < G gates head g for tile t while the compute warps score tile t+1.
     int my_cnt = 0, nkept = 0;
@@ -177,12 +178,11 @@ __global__ void __launch_bounds__(576, 1)
       bool keep = false;
       if (lane < G) {
         const int g = lane;
-        const int w0 = (g / HPG) * WPG;  // the warps that scored head g
-        const float* rm = sRmax + (t & 1) * 16 * GP;
-        float M = rm[w0 * GP + g], sum = sRsum[w0 * GP + g];
-        for (int w = 1; w < WPG; ++w) {
-          M = fmaxf(M, rm[(w0 + w) * GP + g]);
-          sum += sRsum[(w0 + w) * GP + g];
+        const float* rm = sRmax + (t & 1) * NW * GP;
+        float M = rm[g], sum = sRsum[g];
+        for (int w = 1; w < NW; ++w) {
+          M = fmaxf(M, rm[w * GP + g]);
+          sum += sRsum[w * GP + g];
         }
         float l = sL[g] + sum, mu = sM[g];
         keep = (t == 0) || !kGate || (M * p.scale_log2 >= mu + lg2_approx(l) + p.thr);
@@ -224,13 +224,11 @@ __global__ void __launch_bounds__(576, 1)
     }
     named_bar_sync(1, NB);  // C: the last probabilities and sums are written
     if (!aborted && lane < G) {
-      const int g = lane;
-      const int w0 = (g / HPG) * WPG;
       float sum = 0.f;
-      for (int w = 0; w < WPG; ++w) sum += sRsum[(w0 + w) * GP + g];
-      sL[g] += sum;  // fold the last kept tile into the normaliser
+      for (int w = 0; w < NW; ++w) sum += sRsum[w * GP + lane];
+      sL[lane] += sum;  // fold the last kept tile into the normaliser
     }
-    named_bar_sync(1, NB);  // D: the compute warps have summed the key quarters
+    named_bar_sync(1, NB);  // D: the compute warps have summed their partials
     if (!aborted && !abort_raised(fs) && lane < G) {
       const float l = sL[lane];
       p.lse_part[(static_cast<size_t>(b) * p.Hq + hq0 + lane) * p.n_splits + sp_idx] =
@@ -243,163 +241,179 @@ __global__ void __launch_bounds__(576, 1)
   }
 
   // ---------------------------------------------------------- compute warps
+  // Lane (kg, c): key group kg = lane / LPK, 16-byte chunk c = lane % LPK of a
+  // key row. In step s the warp handles keys warp*KPWT + s*KPW + kg. q slices
+  // live in registers; a dot product is reduced across the LPK lanes of a row.
   const float c2 = p.scale_log2;
-  const int kj = tid % BK;             // QK: my key within the tile
-  const int hbase = (tid / BK) * HPG;  // QK: first of my heads
-  const int cp = tid & 63;             // PV: my output column pair
-  const int kq = tid >> 6;             // PV: my slice of the keys
-  float acc[GP][2];
+  const int kg = lane / LPK, c = lane % LPK;
+  float qr[GP][8];
 #pragma unroll
-  for (int g = 0; g < GP; ++g) acc[g][0] = acc[g][1] = 0.f;
-  int nkept = 0;  // kept tiles so far
-  int ndone = 0;  // kept tiles whose PV has run
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qr[g][e] = sq[g * D + c * 8 + e];
+  float acc[GP][8];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+  float ring[NP][STEPS];  // probabilities of pending kept tiles (lane c < GP: head c of its key)
+#pragma unroll
+  for (int i = 0; i < NP; ++i)
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) ring[i][st] = 0.f;
+  int pend = 0, nkept = 0, ndone = 0;
   const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+  const uint32_t chunk_atom = (c >> 3) * (BK * 128), chunk_in = c & 7;
   bool aborted = false;
 
-  auto score = [&](int t, float (&s)[HPG]) {  // s_h = q_h . k_j for my key of tile t and my heads
+  auto row_addr = [&](uint32_t base, int j) { return base + chunk_atom + j * 128 + ((chunk_in ^ (j & 7)) << 4); };
+
+  float sc_cur[STEPS], sc_nxt[STEPS];  // my head's score (lane c < GP) for each step's key
+  auto score = [&](int t, float (&sc)[STEPS]) {
     const int st = t % NK;
     const int kb = t1 - 1 - t;
     const bool okk = mbar_wait_warp(&k_full[st], (t / NK) & 1, fs);
+    float mx[GP];
 #pragma unroll
-    for (int h = 0; h < HPG; ++h) s[h] = 0.f;
-    if (okk && hbase < GP) {
-      const uint32_t rowbase = sKa + st * TB;
-      float part[HPG][4];  // four independent partial sums per head (instruction-level parallelism)
+    for (int g = 0; g < GP; ++g) mx[g] = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < HPG; ++h) part[h][0] = part[h][1] = part[h][2] = part[h][3] = 0.f;
-#pragma unroll 4
-      for (int ch = 0; ch < D / 8; ++ch) {
+    for (int s2 = 0; s2 < STEPS; ++s2) {
+      const int j = warp * KPWT + s2 * KPW + kg;
+      float part[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) part[g] = 0.f;
+      if (okk) {
         uint32_t a0, a1, a2, a3;
-        ld_shared_v4(rowbase + (ch >> 3) * (BK * 128) + sw128_offset(kj, ch & 7), a0, a1, a2, a3);
+        ld_shared_v4(row_addr(sKa + st * TB, j), a0, a1, a2, a3);
         const float kf[8] = {bf16lo_to_f32(a0), bf16hi_to_f32(a0), bf16lo_to_f32(a1), bf16hi_to_f32(a1),
                              bf16lo_to_f32(a2), bf16hi_to_f32(a2), bf16lo_to_f32(a3), bf16hi_to_f32(a3)};
 #pragma unroll
-        for (int h = 0; h < HPG; ++h) {
-          if (hbase + h >= GP) break;
-          const float* qr = sq + (hbase + h) * D + ch * 8;
-          const float4 qa = *reinterpret_cast<const float4*>(qr);
-          const float4 qb = *reinterpret_cast<const float4*>(qr + 4);
-          part[h][0] = fmaf(kf[0], qa.x, part[h][0]); part[h][1] = fmaf(kf[1], qa.y, part[h][1]);
-          part[h][2] = fmaf(kf[2], qa.z, part[h][2]); part[h][3] = fmaf(kf[3], qa.w, part[h][3]);
-          part[h][0] = fmaf(kf[4], qb.x, part[h][0]); part[h][1] = fmaf(kf[5], qb.y, part[h][1]);
-          part[h][2] = fmaf(kf[6], qb.z, part[h][2]); part[h][3] = fmaf(kf[7], qb.w, part[h][3]);
-        }
+        for (int g = 0; g < GP; ++g)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) part[g] = fmaf(kf[e], qr[g][e], part[g]);
       }
 #pragma unroll
-      for (int h = 0; h < HPG; ++h) s[h] = (part[h][0] + part[h][1]) + (part[h][2] + part[h][3]);
+      for (int off = LPK / 2; off > 0; off >>= 1)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
+      const bool live = kb * BK + j < p.Lk;
+      float mine = -INFINITY;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        if (c == g) mine = part[g];
+        if (live) mx[g] = fmaxf(mx[g], part[g]);
+      }
+      sc[s2] = live ? mine : -INFINITY;
     }
     mbar_arrive(&k_empty[st]);  // my reads of this K stage are done
-    const bool live = kb * BK + kj < p.Lk;
 #pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-      float m = live ? s[h] : -INFINITY;
+    for (int off = LPK; off < 32; off <<= 1)
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (lane == 0 && hbase + h < GP) sRmax[((t & 1) * 16 + warp) * GP + hbase + h] = m;
+      for (int g = 0; g < GP; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], off));
+    if (lane < GP) {
+      float v = mx[0];
+#pragma unroll
+      for (int g = 1; g < GP; ++g)
+        if (lane == g) v = mx[g];
+      sRmax[((t & 1) * NW + warp) * GP + lane] = v;
     }
     if (!okk) raise_abort(fs);
   };
 
-  auto run_pv = [&](int n) {  // PV of the n-th kept tile (all compute threads)
+  auto run_pv = [&](const float (&pr)[STEPS]) {  // PV of the oldest pending kept tile
+    const int n = ndone++;
     const int vs = n % NV, ps = n % NP;
     const bool okv = mbar_wait_warp(&v_full[vs], (n / NV) & 1, fs);
-    if (okv && 2 * cp < D) {
+    if (!okv) { aborted = true; return; }
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float al = sAlpha[ps * GP + g];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] *= al;
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < STEPS; ++s2) {
+      const int j = warp * KPWT + s2 * KPW + kg;
+      uint32_t a0, a1, a2, a3;
+      ld_shared_v4(row_addr(sVa + vs * TB, j), a0, a1, a2, a3);
+      const float vf[8] = {bf16lo_to_f32(a0), bf16hi_to_f32(a0), bf16lo_to_f32(a1), bf16hi_to_f32(a1),
+                           bf16lo_to_f32(a2), bf16hi_to_f32(a2), bf16lo_to_f32(a3), bf16hi_to_f32(a3)};
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        const float al = sAlpha[ps * GP + g];
-        acc[g][0] *= al;
-        acc[g][1] *= al;
-      }
-      const int col = 2 * cp;
-      const uint32_t chunk = (col & 63) >> 3;
-      const uint32_t vb = sVa + vs * TB + (col >> 6) * (BK * 128) + ((col & 7) << 1) + kq * KQ * 128;
-      const float* prow = sP + (ps * BK + kq * KQ) * GP;
-#pragma unroll 1
-      for (int m8 = 0; m8 < KQ / 8; ++m8) {
+        const float pg = __shfl_sync(0xffffffffu, pr[s2], kg * LPK + g);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {  // row j = kq*KQ + 8*m8 + r has j % 8 == r
-          const int jl = m8 * 8 + r;
-          uint32_t v2;
-          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v2) : "r"(vb + jl * 128 + ((chunk ^ r) << 4)));
-          const float v0 = bf16lo_to_f32(v2), v1 = bf16hi_to_f32(v2);
-          float pr[GP];
-          if (GP >= 4) {
-#pragma unroll
-            for (int g4 = 0; g4 < GP; g4 += 4) {
-              const float4 x = *reinterpret_cast<const float4*>(prow + jl * GP + g4);
-              pr[g4] = x.x; pr[g4 + 1] = x.y; pr[g4 + 2] = x.z; pr[g4 + 3] = x.w;
-            }
-          } else {
-#pragma unroll
-            for (int g = 0; g < GP; ++g) pr[g] = prow[jl * GP + g];
-          }
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            acc[g][0] = fmaf(pr[g], v0, acc[g][0]);
-            acc[g][1] = fmaf(pr[g], v1, acc[g][1]);
-          }
-        }
+        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
       }
     }
-    if (!okv) aborted = true;
   };
 
-  float s_cur[HPG], s_nxt[HPG];
-  score(0, s_cur);
+  score(0, sc_cur);
   for (int t = 0; t < T; ++t) {
-    const int kb = t1 - 1 - t;
-    named_bar_sync(1, NB);            // A: maxima of tile t are in place
-    if (t + 1 < T) score(t + 1, s_nxt);  // overlaps the gate of tile t
-    named_bar_sync(1, NB);            // B: the decision of tile t is visible
+    named_bar_sync(1, NB);               // A: maxima of tile t are in place
+    if (t + 1 < T) score(t + 1, sc_nxt);  // overlaps the gate of tile t
+    named_bar_sync(1, NB);               // B: the decision of tile t is visible
     const uint32_t flag = *reinterpret_cast<volatile uint32_t*>(sflag);
     if (flag & 2u) { aborted = true; break; }
-    const bool live = kb * BK + kj < p.Lk;
     if (flag & 1u) {  // probabilities of tile t for kept heads, and their per-warp sums
-      float* prow = sP + (nkept % NP) * BK * GP;
+      const bool on = c < GP && sKeep[c < GP ? c : 0] != 0.f;
+      const float mu = sM[c < GP ? c : 0];
+      float pv[STEPS], lsum = 0.f;
 #pragma unroll
-      for (int h = 0; h < HPG; ++h) {
-        const int g = hbase + h;
-        float pv = 0.f;
-        if (g < GP && live && sKeep[g] != 0.f) pv = ex2_approx(fmaf(s_cur[h], c2, -sM[g]));
-        if (g < GP) prow[kj * GP + g] = pv;
-        float sum = pv;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0 && g < GP) sRsum[warp * GP + g] = sum;
+      for (int s2 = 0; s2 < STEPS; ++s2) {
+        pv[s2] = on ? ex2_approx(fmaf(sc_cur[s2], c2, -mu)) : 0.f;
+        lsum += pv[s2];
       }
+#pragma unroll
+      for (int off = LPK; off < 32; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+      if (lane < GP) sRsum[warp * GP + lane] = lsum;
+#pragma unroll
+      for (int i = 0; i + 1 < NP; ++i)
+#pragma unroll
+        for (int s2 = 0; s2 < STEPS; ++s2) ring[i][s2] = ring[i + 1][s2];
+#pragma unroll
+      for (int s2 = 0; s2 < STEPS; ++s2) ring[NP - 1][s2] = pv[s2];
+      ++pend;
       ++nkept;
+      if (pend > kDecLag) {  // the oldest pending tile sits at ring[0]
+        run_pv(ring[0]);
+        --pend;
+      }
     } else {
-#pragma unroll
-      for (int h = 0; h < HPG; ++h)
-        if (lane == 0 && hbase + h < GP) sRsum[warp * GP + hbase + h] = 0.f;
+      if (lane < GP) sRsum[warp * GP + lane] = 0.f;
     }
-    if (nkept - ndone > kDecLag) run_pv(ndone++);  // its P was written at least one barrier ago
 #pragma unroll
-    for (int h = 0; h < HPG; ++h) s_cur[h] = s_nxt[h];
+    for (int s2 = 0; s2 < STEPS; ++s2) sc_cur[s2] = sc_nxt[s2];
   }
 
   named_bar_sync(1, NB);  // C
-  if (!aborted) {
-    while (ndone < nkept) run_pv(ndone++);
-  }
-  named_bar_sync(2, NT);  // compute warps only (barrier 2): every PV read of the rings is done
-  float* ored = reinterpret_cast<float*>(sK);  // [NKQ slices][GP][D], reuses the K ring
-  if (2 * cp < D) {
+  if (!aborted) {  // drain: pending tiles sit at ring[NP - pend .. NP - 1], oldest first
 #pragma unroll
-    for (int g = 0; g < GP; ++g) {
-      ored[(kq * GP + g) * D + 2 * cp] = acc[g][0];
-      ored[(kq * GP + g) * D + 2 * cp + 1] = acc[g][1];
-    }
+    for (int i = 0; i < NP; ++i)
+      if (i >= NP - pend && !aborted) run_pv(ring[i]);
+  }
+  named_bar_sync(2, NT);  // compute warps only (barrier 2): every read of the rings is done
+  float* ored = reinterpret_cast<float*>(sK);  // [NW][GP][D], reuses the K ring
+#pragma unroll
+  for (int off = LPK; off < 32; off <<= 1)  // sum the key groups of the warp
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], off);
+  if (kg == 0) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ored[(warp * GP + g) * D + c * 8 + e] = acc[g][e];
   }
   named_bar_sync(1, NB);  // D (with the gate warp, which has folded the last sums into sL)
   if (!aborted && !abort_raised(fs)) {
     for (int i = tid; i < G * D; i += NT) {
-      const int g = i / D, c = i % D;
+      const int g = i / D, cc = i % D;
       float o = 0.f;
-#pragma unroll
-      for (int x = 0; x < NKQ; ++x) o += ored[(x * GP + g) * D + c];
+#pragma unroll 4
+      for (int x = 0; x < Lay::NPART; ++x) o += ored[(x * GP + g) * D + cc];
       const float l = sL[g];
-      p.o_part[((static_cast<size_t>(b) * p.Hq + hq0 + g) * p.n_splits + sp_idx) * D + c] = l > 0.f ? o / l : 0.f;
+      p.o_part[((static_cast<size_t>(b) * p.Hq + hq0 + g) * p.n_splits + sp_idx) * D + cc] = l > 0.f ? o / l : 0.f;
     }
   }
 }
