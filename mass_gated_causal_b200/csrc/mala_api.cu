@@ -285,11 +285,25 @@ int mala_decode_default_splits(int B, int Hkv, int Lk, int Bk) {
     sms = 148;
   const long long nk = (static_cast<long long>(Lk) + Bk - 1) / Bk;
   const long long units = static_cast<long long>(B) * Hkv;
-  long long s = (16LL * sms + units - 1) / units;  // about 16 CTAs per SM in total
-  s = std::max(1LL, std::min(s, nk));
-  const long long per = (nk + s - 1) / s;  // every split non-empty
-  s = (nk + per - 1) / per;
-  return static_cast<int>(std::min(s, 65535LL));
+  // One decode CTA fills an SM. Pick the split count whose grid takes between
+  // 2 and 8 waves with the fullest last wave, with a small charge per wave
+  // (every CTA pays a pipeline ramp and forces its split's newest tile).
+  long long best = 1;
+  double best_eff = -1.0;
+  for (long long s = 1; s <= std::min(nk, 65535LL); ++s) {
+    const long long per = (nk + s - 1) / s;
+    if ((nk + per - 1) / per != s) continue;  // every split non-empty
+    const double waves = static_cast<double>(units * s) / sms;
+    if (waves > 8.0) break;
+    const double eff = waves / std::ceil(waves);
+    const bool enough = waves >= 2.0;
+    const double score = eff + (enough ? 1.0 : 0.0) - 0.005 * waves;  // each wave costs a pipeline ramp
+    if (score > best_eff + 1e-9) {
+      best_eff = score;
+      best = s;
+    }
+  }
+  return static_cast<int>(best);
 }
 
 int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,

@@ -48,6 +48,35 @@ struct DecParams {
   unsigned* status;
 };
 
+// Sum N per-lane values over the L lanes of a group (lane index c = lane % L,
+// groups aligned to L lanes) so that afterwards lane c holds the group total
+// of value c / (L / N). Each level exchanges half of the values still carried
+// (a reduce-scatter butterfly), so N values take log2(N) + log2(L) - ... fewer
+// shuffles than N full reductions: N = 4, L = 16 needs 5 instead of 16.
+template <int N, int L>
+__device__ __forceinline__ float group_reduce_scatter(float (&v)[N], int c) {
+  int cnt = N;
+#pragma unroll
+  for (int o = L / 2; o >= 1; o >>= 1) {
+    if (cnt > 1) {
+      const bool upper = (c & o) != 0;
+      const int half = cnt / 2;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        if (i < half) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      cnt = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return v[0];
+}
+
 template <int D, int BK, int GP>
 struct DecLayout {
   static constexpr int NK = 3;
@@ -88,7 +117,7 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int NB = NT + 32;        // threads in the per-tile barriers (compute + gate warp)
   static_assert(D == 128 || D == 64, "head dim");
   static_assert(STEPS >= 1 && KPWT % KPW == 0, "tile shape");
-  static_assert(GP <= LPK, "one lane per head within a key row");
+  static_assert(GP <= LPK && LPK % GP == 0, "heads spread evenly over the lanes of a key row");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + Lay::OFF_K;
@@ -246,6 +275,9 @@ __global__ void __launch_bounds__(320, 1)
   // live in registers; a dot product is reduced across the LPK lanes of a row.
   const float c2 = p.scale_log2;
   const int kg = lane / LPK, c = lane % LPK;
+  constexpr int LPH = LPK / GP;  // lanes of a key row that end up holding the same head
+  const int hh = c / LPH;        // the head whose scores this lane holds after the reduction
+  const bool owner = kg == 0 && (c % LPH) == 0;  // writes head hh's per-warp statistics
   float qr[GP][8];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
@@ -256,7 +288,7 @@ __global__ void __launch_bounds__(320, 1)
   for (int g = 0; g < GP; ++g)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-  float ring[NP][STEPS];  // probabilities of pending kept tiles (lane c < GP: head c of its key)
+  float ring[NP][STEPS];  // probabilities of pending kept tiles (head hh of each step's key)
 #pragma unroll
   for (int i = 0; i < NP; ++i)
 #pragma unroll
@@ -268,14 +300,12 @@ __global__ void __launch_bounds__(320, 1)
 
   auto row_addr = [&](uint32_t base, int j) { return base + chunk_atom + j * 128 + ((chunk_in ^ (j & 7)) << 4); };
 
-  float sc_cur[STEPS], sc_nxt[STEPS];  // my head's score (lane c < GP) for each step's key
+  float sc_cur[STEPS], sc_nxt[STEPS];  // head hh's score for each step's key
   auto score = [&](int t, float (&sc)[STEPS]) {
     const int st = t % NK;
     const int kb = t1 - 1 - t;
     const bool okk = mbar_wait_warp(&k_full[st], (t / NK) & 1, fs);
-    float mx[GP];
-#pragma unroll
-    for (int g = 0; g < GP; ++g) mx[g] = -INFINITY;
+    float mx = -INFINITY;  // max over my keys of my head's scores
 #pragma unroll
     for (int s2 = 0; s2 < STEPS; ++s2) {
       const int j = warp * KPWT + s2 * KPW + kg;
@@ -292,31 +322,15 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) part[g] = fmaf(kf[e], qr[g][e], part[g]);
       }
-#pragma unroll
-      for (int off = LPK / 2; off > 0; off >>= 1)
-#pragma unroll
-        for (int g = 0; g < GP; ++g) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
+      const float mine = group_reduce_scatter<GP, LPK>(part, c);  // score of key j for my head hh
       const bool live = kb * BK + j < p.Lk;
-      float mine = -INFINITY;
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        if (c == g) mine = part[g];
-        if (live) mx[g] = fmaxf(mx[g], part[g]);
-      }
+      if (live) mx = fmaxf(mx, mine);
       sc[s2] = live ? mine : -INFINITY;
     }
     mbar_arrive(&k_empty[st]);  // my reads of this K stage are done
 #pragma unroll
-    for (int off = LPK; off < 32; off <<= 1)
-#pragma unroll
-      for (int g = 0; g < GP; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], off));
-    if (lane < GP) {
-      float v = mx[0];
-#pragma unroll
-      for (int g = 1; g < GP; ++g)
-        if (lane == g) v = mx[g];
-      sRmax[((t & 1) * NW + warp) * GP + lane] = v;
-    }
+    for (int off = LPK; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (owner) sRmax[((t & 1) * NW + warp) * GP + hh] = mx;
     if (!okk) raise_abort(fs);
   };
 
@@ -340,7 +354,7 @@ __global__ void __launch_bounds__(320, 1)
                            bf16lo_to_f32(a2), bf16hi_to_f32(a2), bf16lo_to_f32(a3), bf16hi_to_f32(a3)};
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        const float pg = __shfl_sync(0xffffffffu, pr[s2], kg * LPK + g);
+        const float pg = __shfl_sync(0xffffffffu, pr[s2], kg * LPK + g * LPH);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
       }
@@ -355,8 +369,8 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t flag = *reinterpret_cast<volatile uint32_t*>(sflag);
     if (flag & 2u) { aborted = true; break; }
     if (flag & 1u) {  // probabilities of tile t for kept heads, and their per-warp sums
-      const bool on = c < GP && sKeep[c < GP ? c : 0] != 0.f;
-      const float mu = sM[c < GP ? c : 0];
+      const bool on = sKeep[hh] != 0.f;
+      const float mu = sM[hh];
       float pv[STEPS], lsum = 0.f;
 #pragma unroll
       for (int s2 = 0; s2 < STEPS; ++s2) {
@@ -365,7 +379,7 @@ __global__ void __launch_bounds__(320, 1)
       }
 #pragma unroll
       for (int off = LPK; off < 32; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-      if (lane < GP) sRsum[warp * GP + lane] = lsum;
+      if (owner) sRsum[warp * GP + hh] = lsum;
 #pragma unroll
       for (int i = 0; i + 1 < NP; ++i)
 #pragma unroll
@@ -379,7 +393,7 @@ __global__ void __launch_bounds__(320, 1)
         --pend;
       }
     } else {
-      if (lane < GP) sRsum[warp * GP + lane] = 0.f;
+      if (owner) sRsum[warp * GP + hh] = 0.f;
     }
 #pragma unroll
     for (int s2 = 0; s2 < STEPS; ++s2) sc_cur[s2] = sc_nxt[s2];
