@@ -297,7 +297,7 @@ int mala_decode_default_splits(int B, int Hkv, int Lk, int Bk) {
     if (waves > 8.0) break;
     const double eff = waves / std::ceil(waves);
     const bool enough = waves >= 2.0;
-    const double score = eff + (enough ? 1.0 : 0.0) - 0.005 * waves;  // each wave costs a pipeline ramp
+    const double score = eff + (enough ? 1.0 : 0.0) - 0.01 * waves;  // each wave costs a pipeline ramp
     if (score > best_eff + 1e-9) {
       best_eff = score;
       best = s;
