@@ -220,10 +220,13 @@ def run_cuda(args):
     kept_b = torch.empty((B * Hq,), dtype=torch.int32, device=dev)
     ws_bytes = mala.mala_bwd_workspace_size(B, Hq, L, d)
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    fws_bytes = mala.mala_fwd_workspace_size(B, Hkv, L, d)
+    fws = torch.empty((fws_bytes,), dtype=torch.uint8, device=dev)
     nq, nk = -(-L // w.Bq), -(-L // w.Bk)
 
     def step(tau_, km_f=None, km_b=None):
-        rc = mala.mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, kept_f, km_f, stream)
+        rc = mala.mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, fws, fws_bytes, kept_f, km_f,
+                           stream)
         assert rc == 0, mala.mala_status_string(rc)
         rc = mala.mala_bwd(q, k, v, o, do, lse, dq, dk, dv, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, ws,
                            ws_bytes, kept_b, km_b, stream)
@@ -265,7 +268,8 @@ def run_cuda(args):
 
     def train_step(tau_):
         def fn(mid=None):
-            rc = mala.mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, kept_f, None, stream)
+            rc = mala.mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, fws, fws_bytes, kept_f,
+                               None, stream)
             assert rc == 0
             if mid is not None:
                 mid.record(stream)
@@ -369,7 +373,7 @@ def run_cuda(args):
         "e2e": {"value": round(world * step_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roof,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 5 * args.steps,
         "clocks": clocks,
         "peaks": pk,
         "input_gen_s": round(t_gen, 1),

@@ -53,7 +53,8 @@ typedef enum mala_status {
     MALA_ERR_UNSUPPORTED = 2,    /* d, Bq, Bk outside the supported set; pointer not 16-B aligned */
     MALA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than the size query returns */
     MALA_ERR_CUDA = 4,           /* a CUDA runtime / driver call or a launch failed */
-    MALA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait expired (see mala_check_status) */
+    MALA_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait expired (see mala_check_status) */
+    MALA_ERR_RANGE = 6           /* a V value lay outside the fp16 range and was clamped (mala_check_status) */
 } mala_status_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -76,13 +77,18 @@ MALA_API int mala_abi_version(void);
  * row r with a live key satisfies
  *     max_live_j exp(s_rj - m_r) / l_r >= tau / (i_r + 1)      (ties keep).
  * A kept tile updates (m, l) and O for every row of the block; a skipped
- * tile loads no V and does no softmax update and no PV.
+ * tile loads no V and does no softmax update and no PV. The PV product runs in
+ * fp16 on an fp16 copy of V made by the call in `workspace`; V values must lie
+ * inside the fp16 range (|v| <= 65504); larger ones are clamped and reported
+ * as MALA_ERR_RANGE by mala_check_status.
  *
  *   q        [B, L, Hq, d]  bf16, in
  *   k, v     [B, L, Hkv, d] bf16, in
  *   o        [B, L, Hq, d]  bf16, out: O_i = acc_i / l_i
  *   lse      [B, Hq, L]     fp32, out: LSE_i = m_i + ln l_i (natural log)
  *   scale    > 0 (usually 1/sqrt(d)); tau >= 0 (tau = 0: full attention)
+ *   workspace  device scratch of >= mala_fwd_workspace_size(B, Hkv, L, d)
+ *              bytes, 256-byte aligned, caller-owned; contents on entry ignored
  *   kept_tiles [B*Hq] int32, out (required): kept tiles per (b, hq); zeroed
  *            by the call on `stream` before the kernel accumulates into it
  *   keep_map   [B, Hq, nq, nk] uint8, out, nullable (test/debug only): 1 for
@@ -90,8 +96,14 @@ MALA_API int mala_abi_version(void);
  *            tiles are not written. The method itself never reads it.
  */
 MALA_API int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-             int Hkv, int L, int d, float scale, float tau, int Bq, int Bk, int32_t* kept_tiles,
-             uint8_t* keep_map, void* stream);
+             int Hkv, int L, int d, float scale, float tau, int Bq, int Bk, void* workspace,
+             size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
+
+/*
+ * Workspace bytes mala_fwd needs: the fp16 copy of V [B, L, Hkv, d] the PV
+ * product reads (256-byte aligned). Returns 0 for invalid sizes.
+ */
+MALA_API size_t mala_fwd_workspace_size(int B, int Hkv, int L, int d);
 
 /*
  * Workspace bytes mala_bwd needs: an fp32 dQ accumulator [B, L, Hq, d] and
@@ -201,7 +213,8 @@ MALA_API int mala_decode_noalloc(const void* q, const void* kcache, const void* 
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word. Returns MALA_OK, MALA_ERR_DEVICE_TIMEOUT if any kernel since the last
- * check gave up on a bounded wait, or MALA_ERR_CUDA if the stream reports an
+ * check gave up on a bounded wait, MALA_ERR_RANGE if a forward call met a V
+ * value outside the fp16 range, or MALA_ERR_CUDA if the stream reports an
  * error.
  */
 MALA_API int mala_check_status(void* stream);

@@ -31,8 +31,10 @@ MALA_ERR_UNSUPPORTED = 2
 MALA_ERR_WORKSPACE = 3
 MALA_ERR_CUDA = 4
 MALA_ERR_DEVICE_TIMEOUT = 5
+MALA_ERR_RANGE = 6
 
-EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_bwd_workspace_size", "mala_bwd",
+EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_fwd_workspace_size", "mala_bwd_workspace_size",
+            "mala_bwd",
             "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_noalloc_max_bytes",
             "mala_decode_noalloc", "mala_check_status")
 
@@ -40,8 +42,10 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 _lib.mala_status_string.argtypes = [_i]
 _lib.mala_status_string.restype = ctypes.c_char_p
 _lib.mala_abi_version.restype = _i
-_lib.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _vp, _vp]
+_lib.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp, _vp]
 _lib.mala_fwd.restype = _i
+_lib.mala_fwd_workspace_size.argtypes = [_i, _i, _i, _i]
+_lib.mala_fwd_workspace_size.restype = _sz
 _lib.mala_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.mala_bwd_workspace_size.restype = _sz
 _lib.mala_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i,
@@ -99,9 +103,15 @@ def mala_abi_version() -> int:
     return int(_lib.mala_abi_version())
 
 
-def mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, kept_tiles, keep_map=None, stream=None) -> int:
+def mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace, workspace_bytes, kept_tiles,
+             keep_map=None, stream=None) -> int:
     return int(_lib.mala_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), B, Hq, Hkv, L, d, float(scale), float(tau),
-                             Bq, Bk, _p(kept_tiles), _p(keep_map), _stream(stream)))
+                             Bq, Bk, _p(workspace), int(workspace_bytes), _p(kept_tiles), _p(keep_map),
+                             _stream(stream)))
+
+
+def mala_fwd_workspace_size(B, Hkv, L, d) -> int:
+    return int(_lib.mala_fwd_workspace_size(B, Hkv, L, d))
 
 
 def mala_bwd_workspace_size(B, Hq, L, d) -> int:
@@ -146,18 +156,22 @@ def mala_check_status(stream=None) -> int:
 
 
 # ------------------------------------------------------------ conveniences
-def forward(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, keep_map: bool = False, stream=None):
+def forward(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, keep_map: bool = False,
+            workspace=None, stream=None):
     """q [B,L,Hq,d], k/v [B,L,Hkv,d] bf16 CUDA tensors -> (o, lse, kept_tiles, keep_map|None)."""
     import torch
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
+    if workspace is None:
+        workspace = torch.empty((max(1, mala_fwd_workspace_size(B, Hkv, L, d)),), dtype=torch.uint8, device=q.device)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     kept = torch.empty((B * Hq,), dtype=torch.int32, device=q.device)
     km = None
     if keep_map:
         km = torch.full((B, Hq, -(-L // Bq), -(-L // Bk)), 255, dtype=torch.uint8, device=q.device)
-    _check(mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, kept, km, stream), "mala_fwd")
+    _check(mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace,
+                    workspace.numel() * workspace.element_size(), kept, km, stream), "mala_fwd")
     return o, lse, kept, km
 
 

@@ -43,7 +43,8 @@ EncodeTiledFn encode_fn() {
 // Tensor map over a contiguous bf16 BSHD tensor [B, S, H, D] with a
 // {64, 1, rows, 1} box and 128-byte swizzle: one box is a [rows x 64] tile of
 // one head, 128 bytes per row, the layout the UMMA descriptors expect.
-bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int D, int rows) {
+bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int D, int rows,
+                   CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
@@ -52,7 +53,7 @@ bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int 
                            static_cast<cuuint64_t>(S) * H * D * 2};
   cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -96,8 +97,8 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   using Lay = mala::FwdLayout<D, BK>;
   auto kern = mala::mala_fwd_kernel<D, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(p.n_super) * p.B * p.Hq;
-  kern<<<grid, 192, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mo, p);
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * p.B * p.Hq;
+  kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
@@ -165,24 +166,33 @@ const char* mala_status_string(int status) {
     case MALA_ERR_WORKSPACE: return "MALA_ERR_WORKSPACE";
     case MALA_ERR_CUDA: return "MALA_ERR_CUDA";
     case MALA_ERR_DEVICE_TIMEOUT: return "MALA_ERR_DEVICE_TIMEOUT";
+    case MALA_ERR_RANGE: return "MALA_ERR_RANGE";
     default: return "MALA_ERR_UNKNOWN";
   }
 }
 
 int mala_abi_version(void) { return MALA_ABI_VERSION; }
 
+size_t mala_fwd_workspace_size(int B, int Hkv, int L, int d) {
+  if (B < 1 || Hkv < 1 || L < 1 || (d != 64 && d != 128)) return 0;
+  return align256(static_cast<size_t>(B) * L * Hkv * d * 2);
+}
+
 int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int L,
-             int d, float scale, float tau, int Bq, int Bk, int32_t* kept_tiles, uint8_t* keep_map,
-             void* stream) {
+             int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
+             int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
   if (!q || !k || !v || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
   int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
   if (rc != MALA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return MALA_ERR_UNSUPPORTED;
+  const size_t need = mala_fwd_workspace_size(B, Hkv, L, d);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap mq, mk, mv, mo;
   if (!make_bshd_map(&mq, q, B, L, Hq, d, 128) || !make_bshd_map(&mk, k, B, L, Hkv, d, Bk) ||
-      !make_bshd_map(&mv, v, B, L, Hkv, d, Bk) || !make_bshd_map(&mo, o, B, L, Hq, d, 128))
+      !make_bshd_map(&mv, workspace, B, L, Hkv, d, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_bshd_map(&mo, o, B, L, Hq, d, 128))
     return MALA_ERR_CUDA;
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
@@ -190,7 +200,7 @@ int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
   p.nq = (L + Bq - 1) / Bq;
   p.nk = (L + Bk - 1) / Bk;
-  p.n_super = (L + 127) / 128;
+  p.n_pairs = (L + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;
   p.lse = lse;
@@ -198,6 +208,11 @@ int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.keep_map = keep_map;
   p.status = status;
   if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
+  const long long n8 = static_cast<long long>(B) * L * Hkv * d / 8;
+  const int cv_grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
+  mala::mala_v_to_f16_kernel<<<cv_grid, 256, 0, st>>>(static_cast<const uint4*>(v), static_cast<uint4*>(workspace),
+                                                      n8, status);
+  if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
   const bool gate = tau > 0.f;
   if (d == 128 && Bk == 128) return launch_fwd_gate<128, 128>(gate, mq, mk, mv, mo, p, st);
   if (d == 64 && Bk == 128) return launch_fwd_gate<64, 128>(gate, mq, mk, mv, mo, p, st);
@@ -370,7 +385,7 @@ int mala_check_status(void* stream) {
   if (h != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_mala_status, &zero, sizeof(zero)) != cudaSuccess) return MALA_ERR_CUDA;
-    return MALA_ERR_DEVICE_TIMEOUT;
+    return (h & mala::kStatusTimeout) ? MALA_ERR_DEVICE_TIMEOUT : MALA_ERR_RANGE;
   }
   return MALA_OK;
 }

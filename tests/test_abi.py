@@ -29,7 +29,8 @@ def test_header_symbols_exported():
 def test_status_strings_and_version():
     assert mala.mala_abi_version() == 1
     for code, name in ((0, "MALA_OK"), (1, "MALA_ERR_INVALID_ARG"), (2, "MALA_ERR_UNSUPPORTED"),
-                       (3, "MALA_ERR_WORKSPACE"), (4, "MALA_ERR_CUDA"), (5, "MALA_ERR_DEVICE_TIMEOUT")):
+                       (3, "MALA_ERR_WORKSPACE"), (4, "MALA_ERR_CUDA"), (5, "MALA_ERR_DEVICE_TIMEOUT"),
+                       (6, "MALA_ERR_RANGE")):
         assert mala.mala_status_string(code) == name
     assert mala.mala_status_string(99) == "MALA_ERR_UNKNOWN"
 
@@ -39,7 +40,7 @@ P = 256  # a fake, 256-byte aligned "device pointer": never dereferenced by the 
 
 def fwd(**kw):
     a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=1, L=100, d=128, scale=0.1, tau=1.0, Bq=128, Bk=128,
-             kept_tiles=P, keep_map=None, stream=S)
+             workspace=P, workspace_bytes=1 << 30, kept_tiles=P, keep_map=None, stream=S)
     a.update(kw)
     return mala.mala_fwd(**a)
 
@@ -49,6 +50,7 @@ def fwd(**kw):
     (dict(B=0), 1), (dict(L=0), 1), (dict(Hq=3, Hkv=2), 1),
     (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(tau=-1.0), 1), (dict(tau=float("inf")), 1),
     (dict(d=96), 2), (dict(Bq=64, Bk=128), 2), (dict(Bq=32, Bk=32), 2), (dict(q=P + 8), 2),
+    (dict(workspace=None), 3), (dict(workspace_bytes=100), 3), (dict(workspace=P + 16), 3),
 ])
 def test_fwd_rejects(kw, code):
     assert fwd(**kw) == code
@@ -67,6 +69,12 @@ def bwd(**kw):
 ])
 def test_bwd_rejects(kw, code):
     assert bwd(**kw) == code
+
+
+def test_fwd_workspace_size():
+    a256 = lambda x: (x + 255) // 256 * 256
+    assert mala.mala_fwd_workspace_size(2, 4, 1000, 128) == a256(2 * 1000 * 4 * 128 * 2)
+    assert mala.mala_fwd_workspace_size(2, 4, 1000, 96) == 0
 
 
 def test_bwd_workspace_size():
