@@ -295,20 +295,26 @@ __global__ void __launch_bounds__(320, 1)
       local_abort |= !ok;
       tc_fence_after();
       const bool diag = kb * BK + BK - 1 > row0;
+      // first pass (row max): all loads of the S row in flight at once, one wait
       float M = -INFINITY;
-      if (ok) {
+      {
+        uint32_t sv[BK];
 #pragma unroll
-        for (int ch = 0; ch < BK / 32; ++ch) {
-          tmem_ld32(tS + ch * 32, r);
-          tmem_ld_wait();
+        for (int ch = 0; ch < BK / 32; ++ch) tmem_ld32_at(tS + ch * 32, sv + ch * 32);
+        tmem_ld_wait();
+        if (ok) {
+          float mp[8];  // eight independent partial maxima (short dependency chains)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
           if (!diag) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) M = fmaxf(M, __uint_as_float(r[j]));
+            for (int j = 0; j < BK; ++j) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(sv[j]));
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (kb * BK + ch * 32 + j <= row) M = fmaxf(M, __uint_as_float(r[j]));
+            for (int j = 0; j < BK; ++j)
+              if (kb * BK + j <= row) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(sv[j]));
           }
+          M = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         }
       }
       const bool legal = blk_exists && kb <= kbf;
@@ -363,26 +369,45 @@ __global__ void __launch_bounds__(320, 1)
               tmem_st32(tO + ch * 32, r);
             }
           }
-          float rs = 0.f;
+          float rsp[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial row sums
+          const bool plain = !diag && row_ok;   // no masking needed for this row and tile
+          // second pass over S in halves of 64 columns (two loads in flight, one wait each)
 #pragma unroll
-          for (int ch = 0; ch < BK / 32; ++ch) {
-            tmem_ld32(tS + ch * 32, r);
+          for (int hlf = 0; hlf < BK / 64; ++hlf) {
+            uint32_t sh[64];
+            tmem_ld32_at(tS + hlf * 64, sh);
+            tmem_ld32_at(tS + hlf * 64 + 32, sh + 32);
             tmem_ld_wait();
-            uint32_t pk[16];
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              const int key = kb * BK + ch * 32 + 2 * jj;
-              const bool l0 = row_ok && (!diag || key <= row);
-              const bool l1 = row_ok && (!diag || key + 1 <= row);
-              const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(r[2 * jj]), sl2, -m_use)) : 0.f;
-              const float p1 = l1 ? ex2_approx(fmaf(__uint_as_float(r[2 * jj + 1]), sl2, -m_use)) : 0.f;
-              pk[jj] = pack_f16x2(p0, p1);
-              rs += p0 + p1;  // the normaliser sums the fp32 probabilities
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const int ch = hlf * 2 + c2;
+              uint32_t pk[16];
+              if (plain) {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                  const float p0 = ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -m_use));
+                  const float p1 = ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -m_use));
+                  pk[jj] = pack_f16x2(p0, p1);
+                  rsp[jj & 3] += p0 + p1;  // the normaliser sums the fp32 probabilities
+                }
+              } else {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                  const int key = kb * BK + ch * 32 + 2 * jj;
+                  const bool l0 = row_ok && key <= row;
+                  const bool l1 = row_ok && key + 1 <= row;
+                  const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -m_use)) : 0.f;
+                  const float p1 =
+                      l1 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -m_use)) : 0.f;
+                  pk[jj] = pack_f16x2(p0, p1);
+                  rsp[jj & 3] += p0 + p1;
+                }
+              }
+              // P chunk ch covers keys [32ch, 32ch+32) = TMEM columns [16ch, 16ch+16): already read
+              tmem_st16(tS + ch * 16, pk);
             }
-            // P chunk ch covers keys [32ch, 32ch+32) = TMEM columns [16ch, 16ch+16), already read
-            tmem_st16(tS + ch * 16, pk);
           }
-          l += rs;
+          l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
         } else {  // the other query block of this tile keeps it: my rows add nothing
           uint32_t z[16];
 #pragma unroll

@@ -233,6 +233,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// Same as tmem_ld32, into 32 consecutive elements of a larger register array
+// (the offset must be a compile-time constant after unrolling).
+__device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, uint32_t* r) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
