@@ -298,22 +298,27 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t kbits = 0;
       if (kGate) {
         if (ok) {
+          // the whole S^T row: all loads in flight, one wait
+          uint32_t sv[128];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            tmem_ld32(tS + lane_base + ch * 32, r);
-            tmem_ld_wait();
+          for (int ch = 0; ch < 4; ++ch) tmem_ld32_at(tS + lane_base + ch * 32, sv + ch * 32);
+          tmem_ld_wait();
+          bool hit[QPB];
 #pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 th = *reinterpret_cast<const float4*>(vec + 128 + ch * 32 + j4 * 4);
-              const float tv[4] = {th.x, th.y, th.z, th.w};
+          for (int qi = 0; qi < QPB; ++qi) hit[qi] = false;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int il = ch * 32 + j4 * 4 + e;
-                const bool live = !diag || (i0 + il >= kj);
-                if (live && __uint_as_float(r[j4 * 4 + e]) * sl2 >= tv[e]) kbits |= 1u << (il / BQ);
-              }
+          for (int j4 = 0; j4 < 32; ++j4) {
+            const float4 th = *reinterpret_cast<const float4*>(vec + 128 + j4 * 4);
+            const float tv[4] = {th.x, th.y, th.z, th.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int il = j4 * 4 + e;
+              const bool live = !diag || (i0 + il >= kj);
+              hit[il / BQ] |= live && (__uint_as_float(sv[il]) * sl2 >= tv[e]);
             }
           }
+#pragma unroll
+          for (int qi = 0; qi < QPB; ++qi) kbits |= hit[qi] ? (1u << qi) : 0u;
         }
       } else {
 #pragma unroll
@@ -370,24 +375,31 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int qi = 0; qi < QPB; ++qi) qmask |= ((kept >> (qi * 2 + ki)) & 1u) << qi;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        tmem_ld32(tS + lane_base + ch * 32, r);
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t sh[64];
+        tmem_ld32_at(tS + lane_base + hlf * 64, sh);
+        tmem_ld32_at(tS + lane_base + hlf * 64 + 32, sh + 32);
         tmem_ld_wait();
-        uint32_t pk[16];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int il = ch * 32 + 2 * jj;
-          const bool l0 = ((qmask >> (il / BQ)) & 1u) && (!diag || i0 + il >= kj);
-          const bool l1 = ((qmask >> ((il + 1) / BQ)) & 1u) && (!diag || i0 + il + 1 >= kj);
-          const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(r[2 * jj]), sl2, -vec[il])) : 0.f;
-          const float p1 = l1 ? ex2_approx(fmaf(__uint_as_float(r[2 * jj + 1]), sl2, -vec[il + 1])) : 0.f;
-          pk[jj] = pack_bf16x2(p0, p1);
-        }
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int ch = hlf * 2 + c2;
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = ch * 32 + c * 8;
-          st_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pk[4 * c], pk[4 * c + 1],
-                       pk[4 * c + 2], pk[4 * c + 3]);
+          for (int jj = 0; jj < 16; ++jj) {
+            const int il = ch * 32 + 2 * jj;
+            const float2 lv = *reinterpret_cast<const float2*>(vec + il);
+            const bool l0 = ((qmask >> (il / BQ)) & 1u) && (!diag || i0 + il >= kj);
+            const bool l1 = ((qmask >> ((il + 1) / BQ)) & 1u) && (!diag || i0 + il + 1 >= kj);
+            const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -lv.x)) : 0.f;
+            const float p1 = l1 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -lv.y)) : 0.f;
+            pk[jj] = pack_bf16x2(p0, p1);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int col = ch * 32 + c * 8;
+            st_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pk[4 * c],
+                         pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -399,20 +411,23 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       uint32_t dsp[64];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        tmem_ld32(tDP + lane_base + ch * 32, r);
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t dh[64];
+        tmem_ld32_at(tDP + lane_base + hlf * 64, dh);
+        tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, dh + 32);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = ch * 32 + c * 8;
+        for (int c = 0; c < 8; ++c) {
+          const int col = hlf * 64 + c * 8;
           uint32_t pp[4];
           ld_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pp[0], pp[1], pp[2], pp[3]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int il = col + 2 * e;
-            const float d0 = __uint_as_float(r[c * 8 + 2 * e]) - vec[256 + il];
-            const float d1 = __uint_as_float(r[c * 8 + 2 * e + 1]) - vec[256 + il + 1];
-            dsp[ch * 16 + c * 4 + e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * d0, bf16hi_to_f32(pp[e]) * d1);
+            const float2 dv2 = *reinterpret_cast<const float2*>(vec + 256 + il);
+            const float d0 = __uint_as_float(dh[c * 8 + 2 * e]) - dv2.x;
+            const float d1 = __uint_as_float(dh[c * 8 + 2 * e + 1]) - dv2.y;
+            dsp[hlf * 32 + c * 4 + e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * d0, bf16hi_to_f32(pp[e]) * d1);
           }
         }
       }
@@ -434,15 +449,17 @@ __global__ void __launch_bounds__(192, 1)
         float* dst = p.dq_acc + (static_cast<size_t>(b) * p.L + i) * (static_cast<size_t>(p.Hq) * D) +
                      static_cast<size_t>(hq) * D;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          tmem_ld32(tDP + lane_base + ch * 32, r);
+        for (int hlf = 0; hlf < D / 64; ++hlf) {
+          uint32_t qh[64];
+          tmem_ld32_at(tDP + lane_base + hlf * 64, qh);
+          tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, qh + 32);
           tmem_ld_wait();
           if (i < p.L) {
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              red_add_v4(dst + ch * 32 + q4 * 4, p.scale * __uint_as_float(r[q4 * 4]),
-                         p.scale * __uint_as_float(r[q4 * 4 + 1]), p.scale * __uint_as_float(r[q4 * 4 + 2]),
-                         p.scale * __uint_as_float(r[q4 * 4 + 3]));
+            for (int q4 = 0; q4 < 16; ++q4)
+              red_add_v4(dst + hlf * 64 + q4 * 4, p.scale * __uint_as_float(qh[q4 * 4]),
+                         p.scale * __uint_as_float(qh[q4 * 4 + 1]), p.scale * __uint_as_float(qh[q4 * 4 + 2]),
+                         p.scale * __uint_as_float(qh[q4 * 4 + 3]));
           }
         }
       }
