@@ -17,12 +17,16 @@
 // when Bk = 64) of one (b, KV head) and walks the query tiles of every query
 // head of the GQA group, 128 queries at a time, from the diagonal tile to the
 // end. dK and dV accumulate in TMEM across the whole walk.
-//   warps 0-3  thread t owns key row t (TMEM lane t of S^T, dP^T, dK, dV) and,
-//              for the dQ drain, query row t of the tile (TMEM lane t of dQ)
-//   warp  4    producer: K, V once; Q tiles and the per-query LSE / threshold
+//   warps 0-3  compute: thread t owns key row t (TMEM lane t of S^T, dP^T,
+//              dK, dV): gate, P^T, dS^T
+//   warps 4-7  dQ drain: thread t owns query row t of a kept tile (TMEM lane t
+//              of dQ) and reduces it into the fp32 accumulator, while the
+//              compute warps move on to the next tile
+//   warp  8    producer: K, V once; Q tiles and the per-query LSE / threshold
 //              / D vectors through a 2-stage ring
-//   warp  5    MMA issuer: S^T = K Q^T, then for kept tiles the dO TMA,
-//              dP^T = V dO^T, dV += P^T dO, dK += dS^T Q, dQ = dS K
+//   warp  9    MMA issuer: S^T = K Q^T, then for kept tiles the dO TMA,
+//              dP^T = V dO^T, dV += P^T dO, the next tile's S^T, then
+//              dK += dS^T Q and dQ = dS K
 // P^T and dS^T share one shared-memory tile: dS^T overwrites P^T once the dV
 // MMA that reads P^T has finished. dQ reuses the dP^T TMEM columns and is
 // added to the fp32 accumulator with vector reductions.
@@ -59,8 +63,8 @@ struct BwdLayout {
   static constexpr int OFF_VEC = OFF_PS + PS_BYTES;  // [2 stages][LSE2, T, D][128] fp32
   static constexpr int OFF_BAR = OFF_VEC + 2 * 3 * 128 * 4;
   // kv_full, q_full[2], q_empty[2], s_full, st_free, dec, do_full, do_empty,
-  // dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free, ps_free, mma_final
-  static constexpr int N_BARS = 18;
+  // dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free, ps_free, mma_final, info_full
+  static constexpr int N_BARS = 19;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
@@ -74,7 +78,7 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 }
 
 template <int D, int BK, bool kGate>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     mala_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
@@ -111,12 +115,14 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* dq_free = bars + 15;
   uint64_t* ps_free = bars + 16;
   uint64_t* mma_final = bars + 17;
+  uint64_t* info_full = bars + 18;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   uint32_t* tmem_slot = misc + 0;
   int* abort_flag = reinterpret_cast<int*>(misc + 1);
   uint32_t* dec_flags = misc + 2;
-  uint32_t* vote = misc + 4;   // [2][4]
-  uint32_t* evote = misc + 12; // [4]
+  uint32_t* vote = misc + 4;    // [2][4]
+  uint32_t* evote = misc + 12;  // [4]
+  int* info = reinterpret_cast<int*>(misc + 16);  // {hq, i0} of the kept tile the drain warpgroup handles next
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -147,10 +153,11 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(dq_free, 128);
     mbar_init(ps_free, 1);
     mbar_init(mma_final, 1);
+    mbar_init(info_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(tmem_slot, Lay::TMEM_COLS);
     tmem_relinquish();
   }
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(192, 1)
   const FailState fs{abort_flag, p.status};
   const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 256 + D;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * TB);
@@ -200,36 +207,40 @@ __global__ void __launch_bounds__(192, 1)
       for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait_drain(&q_full[t & 1], (t >> 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
       const uint32_t sPSa = smem_u32(sPS);
       int nd = 0;
-      bool ok = mbar_wait(kv_full, 0, fs);
+      auto issue_qk = [&](int st) {  // S^T = K Q^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16_ss(tS, sdesc_sw128(sKa + off, 16, 1024), sdesc_sw128(sQa + st * TB + off, 16, 1024), IDESC_S,
+                       kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+      };
+      bool ok = mbar_wait(kv_full, 0, fs) && mbar_wait(&q_full[0], 0, fs);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+      }
       for (int t = 0; ok && t < T; ++t) {
         const int st = t & 1;
         const int hq = hkv * p.G + t / nqs;
         const int i0 = (ks + t % nqs) * 128;
         const uint32_t sQs = sQa + st * TB;
-        if (!mbar_wait(&q_full[st], (t >> 1) & 1, fs)) break;
-        if (t >= 1 && !mbar_wait(st_free, (t - 1) & 1, fs)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(tS, sdesc_sw128(sKa + off, 16, 1024), sdesc_sw128(sQs + off, 16, 1024), IDESC_S,
-                       kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full);
         if (!mbar_wait(dec_bar, t & 1, fs)) break;
         const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(dec_flags);
         if (dec & kBwdAbort) break;
-        if (dec & kBwdAny) {
+        const bool keep = (dec & kBwdAny) != 0;
+        if (keep) {
           if (nd >= 1 && !mbar_wait(do_empty, (nd - 1) & 1, fs)) break;
           mbar_arrive_expect_tx(do_full, TB);
           for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, i0, b);
-          if (nd >= 1 && !mbar_wait(dq_free, (nd - 1) & 1, fs)) break;
+          if (nd >= 1 && !mbar_wait(dq_free, (nd - 1) & 1, fs)) break;  // dQ(nd-1) drained from the dP^T columns
           if (!mbar_wait(do_full, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
@@ -249,6 +260,14 @@ __global__ void __launch_bounds__(192, 1)
           }
           umma_commit(do_empty);
           umma_commit(dv_done);
+        }
+        if (t + 1 < T) {  // the next tile's scores as early as possible
+          if (!mbar_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, fs)) break;
+          if (!mbar_wait(st_free, t & 1, fs)) break;  // S^T(t) consumed
+          tc_fence_after();
+          issue_qk((t + 1) & 1);
+        }
+        if (keep) {
           if (!mbar_wait(ds_ready, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
@@ -265,16 +284,56 @@ __global__ void __launch_bounds__(192, 1)
           }
           umma_commit(dq_full);
           umma_commit(ps_free);
+          info[0] = hq;  // the drain warpgroup finished dQ(nd-1) before dP(nd) was issued
+          info[1] = i0;
+          mbar_arrive(info_full);
           ++nd;
         }
-        umma_commit(&q_empty[st]);
+        umma_commit(&q_empty[st]);  // Q(t): QK(t) and dK(t) issued
       }
+      // tell the drain warpgroup there is nothing more, once it has taken the last tile
+      if (nd >= 1) mbar_wait(dq_free, (nd - 1) & 1, fs);
+      info[0] = -1;
+      mbar_arrive(info_full);
       umma_commit(mma_final);
       if (nd >= 1) mbar_wait_drain(do_full, (nd - 1) & 1);
     }
     __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ dQ drain warpgroup
+    // Query row tid of each kept tile: TMEM lane tid of the dQ accumulator, added
+    // to the fp32 workspace with vector reductions.
+    const int tid = threadIdx.x - 128;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    for (int n = 0;; ++n) {
+      if (!mbar_wait_warp(info_full, n & 1, fs)) break;
+      const int hq = *reinterpret_cast<volatile int*>(&info[0]);
+      const int i0 = *reinterpret_cast<volatile int*>(&info[1]);
+      if (hq < 0) break;
+      if (!mbar_wait_warp(dq_full, n & 1, fs)) break;
+      tc_fence_after();
+      const int i = i0 + tid;
+      float* dst = p.dq_acc + (static_cast<size_t>(b) * p.L + i) * (static_cast<size_t>(p.Hq) * D) +
+                   static_cast<size_t>(hq) * D;
+#pragma unroll
+      for (int hlf = 0; hlf < D / 64; ++hlf) {
+        uint32_t qh[64];
+        tmem_ld32_at(tDP + lane_base + hlf * 64, qh);
+        tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, qh + 32);
+        tmem_ld_wait();
+        if (i < p.L) {
+#pragma unroll
+          for (int q4 = 0; q4 < 16; ++q4)
+            red_add_v4(dst + hlf * 64 + q4 * 4, p.scale * __uint_as_float(qh[q4 * 4]),
+                       p.scale * __uint_as_float(qh[q4 * 4 + 1]), p.scale * __uint_as_float(qh[q4 * 4 + 2]),
+                       p.scale * __uint_as_float(qh[q4 * 4 + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
   } else {
-    // ------------------------------------------------------------ compute warps
+    // ------------------------------------------------------------ compute warpgroup
     const int tid = threadIdx.x;
     const int kj = k0 + tid;  // my key
     const int ki = tid / BK;  // my key block inside the CTA
@@ -291,35 +350,37 @@ __global__ void __launch_bounds__(192, 1)
       const int qs = ks + t % nqs;
       const int i0 = qs * 128;
       const bool diag = qs == ks;
-      const float* vec = sVec + st * 384;
+      const uint32_t vec_s = smem_u32(sVec + st * 384);  // LSE2 | gate threshold | D, 128 each
       const bool ok = mbar_wait_warp(s_full, t & 1, fs);
       local_abort |= !ok;
       tc_fence_after();
       uint32_t kbits = 0;
       if (kGate) {
-        if (ok) {
-          // the whole S^T row: all loads in flight, one wait
-          uint32_t sv[128];
+        bool hit[QPB];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) tmem_ld32_at(tS + lane_base + ch * 32, sv + ch * 32);
+        for (int qi = 0; qi < QPB; ++qi) hit[qi] = false;
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {  // S^T row in halves: two loads in flight, one wait
+          uint32_t sh[64];
+          tmem_ld32_at(tS + lane_base + hlf * 64, sh);
+          tmem_ld32_at(tS + lane_base + hlf * 64 + 32, sh + 32);
           tmem_ld_wait();
-          bool hit[QPB];
+          if (ok) {
 #pragma unroll
-          for (int qi = 0; qi < QPB; ++qi) hit[qi] = false;
+            for (int j4 = 0; j4 < 16; ++j4) {
+              const float4 th = ld_shared_f4(vec_s + 4 * (128 + hlf * 64 + j4 * 4));
+              const float tv[4] = {th.x, th.y, th.z, th.w};
 #pragma unroll
-          for (int j4 = 0; j4 < 32; ++j4) {
-            const float4 th = *reinterpret_cast<const float4*>(vec + 128 + j4 * 4);
-            const float tv[4] = {th.x, th.y, th.z, th.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int il = j4 * 4 + e;
-              const bool live = !diag || (i0 + il >= kj);
-              hit[il / BQ] |= live && (__uint_as_float(sv[il]) * sl2 >= tv[e]);
+              for (int e = 0; e < 4; ++e) {
+                const int il = hlf * 64 + j4 * 4 + e;
+                const bool live = !diag || (i0 + il >= kj);
+                hit[il / BQ] |= live && (__uint_as_float(sh[j4 * 4 + e]) * sl2 >= tv[e]);
+              }
             }
           }
-#pragma unroll
-          for (int qi = 0; qi < QPB; ++qi) kbits |= hit[qi] ? (1u << qi) : 0u;
         }
+#pragma unroll
+        for (int qi = 0; qi < QPB; ++qi) kbits |= hit[qi] ? (1u << qi) : 0u;
       } else {
 #pragma unroll
         for (int qi = 0; qi < QPB; ++qi) {
@@ -387,11 +448,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int il = ch * 32 + 2 * jj;
-            const float2 lv = *reinterpret_cast<const float2*>(vec + il);
+            const float2 lv = ld_shared_f2(vec_s + 4 * il);
             const bool l0 = ((qmask >> (il / BQ)) & 1u) && (!diag || i0 + il >= kj);
             const bool l1 = ((qmask >> ((il + 1) / BQ)) & 1u) && (!diag || i0 + il + 1 >= kj);
-            const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -lv.x)) : 0.f;
-            const float p1 = l1 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -lv.y)) : 0.f;
+            // dead entries go through ex2 as -inf (-> 0): no branch around the inline asm
+            const float p0 = ex2_approx(l0 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -lv.x) : -INFINITY);
+            const float p1 = ex2_approx(l1 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -lv.y) : -INFINITY);
             pk[jj] = pack_bf16x2(p0, p1);
           }
 #pragma unroll
@@ -406,10 +468,10 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(p_ready);
       mbar_arrive(st_free);
-      // ---- dS^T = P^T * (dP^T - D)
+      // ---- dS^T = P^T * (dP^T - D), written over P^T once the dV MMA has read it
       local_abort |= !mbar_wait_warp(dp_full, nd & 1, fs);
+      local_abort |= !mbar_wait_warp(dv_done, nd & 1, fs);
       tc_fence_after();
-      uint32_t dsp[64];
 #pragma unroll
       for (int hlf = 0; hlf < 2; ++hlf) {
         uint32_t dh[64];
@@ -419,52 +481,23 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const int col = hlf * 64 + c * 8;
-          uint32_t pp[4];
-          ld_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pp[0], pp[1], pp[2], pp[3]);
+          const uint32_t addr = sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3);
+          uint32_t pp[4], ds[4];
+          ld_shared_v4(addr, pp[0], pp[1], pp[2], pp[3]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int il = col + 2 * e;
-            const float2 dv2 = *reinterpret_cast<const float2*>(vec + 256 + il);
+            const float2 dv2 = ld_shared_f2(vec_s + 4 * (256 + il));
             const float d0 = __uint_as_float(dh[c * 8 + 2 * e]) - dv2.x;
             const float d1 = __uint_as_float(dh[c * 8 + 2 * e + 1]) - dv2.y;
-            dsp[hlf * 32 + c * 4 + e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * d0, bf16hi_to_f32(pp[e]) * d1);
+            ds[e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * d0, bf16hi_to_f32(pp[e]) * d1);
           }
+          st_shared_v4(addr, ds[0], ds[1], ds[2], ds[3]);
         }
-      }
-      local_abort |= !mbar_wait_warp(dv_done, nd & 1, fs);  // the dV MMA has read P^T
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int col = c * 8;
-        st_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), dsp[4 * c], dsp[4 * c + 1],
-                     dsp[4 * c + 2], dsp[4 * c + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_ready);
-      // ---- dQ rows of this tile: fp32 reductions into the accumulator
-      local_abort |= !mbar_wait_warp(dq_full, nd & 1, fs);
-      tc_fence_after();
-      {
-        const int i = i0 + tid;
-        float* dst = p.dq_acc + (static_cast<size_t>(b) * p.L + i) * (static_cast<size_t>(p.Hq) * D) +
-                     static_cast<size_t>(hq) * D;
-#pragma unroll
-        for (int hlf = 0; hlf < D / 64; ++hlf) {
-          uint32_t qh[64];
-          tmem_ld32_at(tDP + lane_base + hlf * 64, qh);
-          tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, qh + 32);
-          tmem_ld_wait();
-          if (i < p.L) {
-#pragma unroll
-            for (int q4 = 0; q4 < 16; ++q4)
-              red_add_v4(dst + hlf * 64 + q4 * 4, p.scale * __uint_as_float(qh[q4 * 4]),
-                         p.scale * __uint_as_float(qh[q4 * 4 + 1]), p.scale * __uint_as_float(qh[q4 * 4 + 2]),
-                         p.scale * __uint_as_float(qh[q4 * 4 + 3]));
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(dq_free);
       ++nd;
     }
 
@@ -517,7 +550,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) mbar_wait_drain(mma_final, 0);
     __syncwarp();
     tc_fence_after();

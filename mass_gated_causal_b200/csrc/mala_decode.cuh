@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(320, 1)
       float pv[STEPS], lsum = 0.f;
 #pragma unroll
       for (int s2 = 0; s2 < STEPS; ++s2) {
-        pv[s2] = on ? ex2_approx(fmaf(sc_cur[s2], c2, -mu)) : 0.f;
+        pv[s2] = ex2_approx(on ? fmaf(sc_cur[s2], c2, -mu) : -INFINITY);  // no branch around the asm
         lsum += pv[s2];
       }
 #pragma unroll

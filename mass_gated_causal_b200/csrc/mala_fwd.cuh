@@ -396,9 +396,10 @@ __global__ void __launch_bounds__(320, 1)
                   const int key = kb * BK + ch * 32 + 2 * jj;
                   const bool l0 = row_ok && key <= row;
                   const bool l1 = row_ok && key + 1 <= row;
-                  const float p0 = l0 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -m_use)) : 0.f;
+                  // masked entries go through ex2 as -inf (-> 0): no branch around the inline asm
+                  const float p0 = ex2_approx(l0 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -m_use) : -INFINITY);
                   const float p1 =
-                      l1 ? ex2_approx(fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -m_use)) : 0.f;
+                      ex2_approx(l1 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -m_use) : -INFINITY);
                   pk[jj] = pack_f16x2(p0, p1);
                   rsp[jj & 3] += p0 + p1;
                 }
