@@ -59,6 +59,23 @@ bool make_bshd_map(CUtensorMap* map, const void* base, int B, int S, int H, int 
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over the fp32 dQ accumulator [B, S, H, D] with a {32, 1, 32, 1}
+// box and 128-byte swizzle: a [32 rows x 32] fp32 block of one head.
+bool make_dq_acc_map(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H) * D * 4,
+                           static_cast<cuuint64_t>(S) * H * D * 4};
+  cuuint32_t box[4] = {32, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
@@ -111,21 +128,22 @@ int launch_fwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, con
 // --------------------------------------------------------------- backward
 template <int D, int BK, bool G>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-               const CUtensorMap& mdk, const CUtensorMap& mdv, const mala::BwdParams& p, cudaStream_t st) {
+               const CUtensorMap& mdk, const CUtensorMap& mdv, const CUtensorMap& mdq, const mala::BwdParams& p,
+               cudaStream_t st) {
   using Lay = mala::BwdLayout<D>;
   auto kern = mala::mala_bwd_kernel<D, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.n_super) * p.B * p.Hkv;
-  kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, p);
+  kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
 template <int D, int BK>
 int launch_bwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
-                    const mala::BwdParams& p, cudaStream_t st) {
-  return gate ? launch_bwd<D, BK, true>(mq, mk, mv, mdo, mdk, mdv, p, st)
-              : launch_bwd<D, BK, false>(mq, mk, mv, mdo, mdk, mdv, p, st);
+                    const CUtensorMap& mdq, const mala::BwdParams& p, cudaStream_t st) {
+  return gate ? launch_bwd<D, BK, true>(mq, mk, mv, mdo, mdk, mdv, mdq, p, st)
+              : launch_bwd<D, BK, false>(mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
 }
 
 // ----------------------------------------------------------------- decode
@@ -246,6 +264,8 @@ int mala_bwd(const void* q, const void* k, const void* v, const void* o, const v
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
   float* dq_acc = static_cast<float*>(workspace);
+  CUtensorMap mdq;
+  if (!make_dq_acc_map(&mdq, dq_acc, B, L, Hq, d)) return MALA_ERR_CUDA;
   float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                          align256(static_cast<size_t>(B) * L * Hq * d * 4));
   mala::BwdParams p;
@@ -274,10 +294,10 @@ int mala_bwd(const void* q, const void* k, const void* v, const void* o, const v
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
 
   const bool gate = tau > 0.f;
-  if (d == 128 && Bk == 128) rc = launch_bwd_gate<128, 128>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
-  else if (d == 64 && Bk == 128) rc = launch_bwd_gate<64, 128>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
-  else if (d == 128 && Bk == 64) rc = launch_bwd_gate<128, 64>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
-  else rc = launch_bwd_gate<64, 64>(gate, mq, mk, mv, mdo, mdk, mdv, p, st);
+  if (d == 128 && Bk == 128) rc = launch_bwd_gate<128, 128>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  else if (d == 64 && Bk == 128) rc = launch_bwd_gate<64, 128>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  else if (d == 128 && Bk == 64) rc = launch_bwd_gate<128, 64>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  else rc = launch_bwd_gate<64, 64>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
   if (rc != MALA_OK) return rc;
 
   const long long n8 = static_cast<long long>(B) * L * Hq * d / 8;

@@ -42,7 +42,7 @@ struct BwdParams {
   float scale, scale_log2, log2_tau;
   const float* lse;   // [B, Hq, L]
   const float* dvec;  // [B, Hq, L]: D_i
-  float* dq_acc;      // [B, L, Hq, d] fp32
+  float* dq_acc;      // [B, L, Hq, d] fp32 (the kernel adds into it through its tensor map)
   int32_t* kept_tiles;
   uint8_t* keep_map;
   unsigned* status;
@@ -60,29 +60,26 @@ struct BwdLayout {
   static constexpr int OFF_Q = OFF_V + T_BYTES;  // 2 stages
   static constexpr int OFF_DO = OFF_Q + 2 * T_BYTES;
   static constexpr int OFF_PS = OFF_DO + T_BYTES;
-  static constexpr int OFF_VEC = OFF_PS + PS_BYTES;  // [2 stages][LSE2, T, D][128] fp32
+  static constexpr int STG_WARP = 32 * 32 * 4;  // dQ staging: [32 rows x 32] fp32 per drain warp
+  static constexpr int OFF_STG = OFF_PS + PS_BYTES;  // 1024-aligned (128-byte swizzle)
+  static constexpr int OFF_VEC = OFF_STG + 4 * STG_WARP;  // [2 stages][LSE2, T, D][128] fp32
   static constexpr int OFF_BAR = OFF_VEC + 2 * 3 * 128 * 4;
   // kv_full, q_full[2], q_empty[2], s_full, st_free, dec, do_full, do_empty,
   // dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free, ps_free, mma_final, info_full
   static constexpr int N_BARS = 19;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-  static constexpr int BYTES = OFF_MISC + 64;
+  static constexpr int BYTES = OFF_MISC + 96;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
   static constexpr int TMEM_COLS = 512;  // S^T 128 | dP^T/dQ 128 | dK D | dV D
   static_assert(ALLOC_BYTES <= 232448, "backward shared memory exceeds the per-CTA limit");
 };
-
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 template <int D, int BK, bool kGate>
 __global__ void __launch_bounds__(320, 1)
     mala_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Lay = BwdLayout<D>;
   constexpr int BQ = BK, QPB = 128 / BQ, KPB = 128 / BK;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
@@ -301,10 +298,15 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dQ drain warpgroup
-    // Query row tid of each kept tile: TMEM lane tid of the dQ accumulator, added
-    // to the fp32 workspace with vector reductions.
-    const int tid = threadIdx.x - 128;
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // Warp w owns query rows [32w, 32w+32) of each kept tile (TMEM lanes of the
+    // dQ accumulator). It reads its rows out of TMEM, hands the columns back to
+    // the MMA issuer, and adds them to the fp32 workspace 32 columns at a time:
+    // a swizzled [32 x 32] fp32 block in shared memory, reduced into global
+    // memory by one TMA add (whole 128-byte lines, element-wise atomic adds).
+    const int wq = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    uint8_t* stg = smem + Lay::OFF_STG + wq * Lay::STG_WARP;
+    const uint32_t stg_s = smem_u32(stg);
     for (int n = 0;; ++n) {
       if (!mbar_wait_warp(info_full, n & 1, fs)) break;
       const int hq = *reinterpret_cast<volatile int*>(&info[0]);
@@ -312,26 +314,33 @@ __global__ void __launch_bounds__(320, 1)
       if (hq < 0) break;
       if (!mbar_wait_warp(dq_full, n & 1, fs)) break;
       tc_fence_after();
-      const int i = i0 + tid;
-      float* dst = p.dq_acc + (static_cast<size_t>(b) * p.L + i) * (static_cast<size_t>(p.Hq) * D) +
-                   static_cast<size_t>(hq) * D;
+      uint32_t qh[D];
 #pragma unroll
-      for (int hlf = 0; hlf < D / 64; ++hlf) {
-        uint32_t qh[64];
-        tmem_ld32_at(tDP + lane_base + hlf * 64, qh);
-        tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, qh + 32);
-        tmem_ld_wait();
-        if (i < p.L) {
-#pragma unroll
-          for (int q4 = 0; q4 < 16; ++q4)
-            red_add_v4(dst + hlf * 64 + q4 * 4, p.scale * __uint_as_float(qh[q4 * 4]),
-                       p.scale * __uint_as_float(qh[q4 * 4 + 1]), p.scale * __uint_as_float(qh[q4 * 4 + 2]),
-                       p.scale * __uint_as_float(qh[q4 * 4 + 3]));
-        }
-      }
+      for (int c = 0; c < D / 32; ++c) tmem_ld32_at(tDP + lane_base + c * 32, qh + c * 32);
+      tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(dq_free);
+      const int row0 = i0 + wq * 32;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        if (lane == 0) bulk_wait_read0();  // the previous block has left the staging buffer
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(stg_s + sw128_offset(lane, j), __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j])),
+                       __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j + 1])),
+                       __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j + 2])),
+                       __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j + 3])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < p.L) {  // rows at or past L are clipped by the tensor map
+          tma_reduce_add_4d(&tm_dq, stg, c * 32, hq, row0, b);
+          bulk_commit();
+        }
+      }
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ compute warpgroup
     const int tid = threadIdx.x;
