@@ -17,19 +17,21 @@
 // when Bk = 64) of one (b, KV head) and walks the query tiles of every query
 // head of the GQA group, 128 queries at a time, from the diagonal tile to the
 // end. dK and dV accumulate in TMEM across the whole walk.
-//   warps 0-3  compute: thread t owns key row t (TMEM lane t of S^T, dP^T,
-//              dK, dV): gate, P^T, dS^T
+//   warps 0-3  compute: thread t owns query row t of the current tile (TMEM
+//              lane t of S and dP), so its LSE, gate threshold and D are
+//              scalars: gate, P, dS; at the end, key row t of dK and dV
 //   warps 4-7  dQ drain: thread t owns query row t of a kept tile (TMEM lane t
-//              of dQ) and reduces it into the fp32 accumulator, while the
-//              compute warps move on to the next tile
+//              of dQ) and adds it to the fp32 accumulator, while the compute
+//              warps move on to the next tile
 //   warp  8    producer: K, V once; Q tiles and the per-query LSE / threshold
 //              / D vectors through a 2-stage ring
-//   warp  9    MMA issuer: S^T = K Q^T, then for kept tiles the dO TMA,
-//              dP^T = V dO^T, dV += P^T dO, the next tile's S^T, then
+//   warp  9    MMA issuer: S = Q K^T, then for kept tiles the dO TMA,
+//              dP = dO V^T, dV += P^T dO, the next tile's S, then
 //              dK += dS^T Q and dQ = dS K
-// P^T and dS^T share one shared-memory tile: dS^T overwrites P^T once the dV
-// MMA that reads P^T has finished. dQ reuses the dP^T TMEM columns and is
-// added to the fp32 accumulator with vector reductions.
+// P and dS share one shared-memory tile (query rows, 128-byte swizzle): dS
+// overwrites P once the dV MMA that reads P^T (MN-major) has finished. dQ
+// reuses the dP TMEM columns and is added to the fp32 accumulator by TMA
+// reduce-add.
 #pragma once
 
 #include "mala_ptx.cuh"
@@ -70,7 +72,7 @@ struct BwdLayout {
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 96;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
-  static constexpr int TMEM_COLS = 512;  // S^T 128 | dP^T/dQ 128 | dK D | dV D
+  static constexpr int TMEM_COLS = 512;  // S 128 | dP/dQ 128 | dK D | dV D
   static_assert(ALLOC_BYTES <= 232448, "backward shared memory exceeds the per-CTA limit");
 };
 
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int BQ = BK, QPB = 128 / BQ, KPB = 128 / BK;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
   constexpr uint32_t IDESC_KN = idesc_bf16(128, D, false, true);  // A K-major, B MN-major
-  constexpr uint32_t IDESC_DQ = idesc_bf16(128, D, true, true);   // A, B MN-major
+  constexpr uint32_t IDESC_MN = idesc_bf16(128, D, true, true);   // A, B MN-major
   constexpr int TB = Lay::T_BYTES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -210,11 +212,11 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
       const uint32_t sPSa = smem_u32(sPS);
       int nd = 0;
-      auto issue_qk = [&](int st) {  // S^T = K Q^T
+      auto issue_qk = [&](int st) {  // S = Q K^T
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(tS, sdesc_sw128(sKa + off, 16, 1024), sdesc_sw128(sQa + st * TB + off, 16, 1024), IDESC_S,
+          umma_bf16_ss(tS, sdesc_sw128(sQa + st * TB + off, 16, 1024), sdesc_sw128(sKa + off, 16, 1024), IDESC_S,
                        kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full);
@@ -237,30 +239,30 @@ __global__ void __launch_bounds__(320, 1)
           if (nd >= 1 && !mbar_wait(do_empty, (nd - 1) & 1, fs)) break;
           mbar_arrive_expect_tx(do_full, TB);
           for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, i0, b);
-          if (nd >= 1 && !mbar_wait(dq_free, (nd - 1) & 1, fs)) break;  // dQ(nd-1) drained from the dP^T columns
+          if (nd >= 1 && !mbar_wait(dq_free, (nd - 1) & 1, fs)) break;  // dQ(nd-1) drained from the dP columns
           if (!mbar_wait(do_full, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+          for (int kk = 0; kk < D / 16; ++kk) {  // dP = dO V^T
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16_ss(tDP, sdesc_sw128(sVa + off, 16, 1024), sdesc_sw128(sDOa + off, 16, 1024), IDESC_S,
+            umma_bf16_ss(tDP, sdesc_sw128(sDOa + off, 16, 1024), sdesc_sw128(sVa + off, 16, 1024), IDESC_S,
                          kk > 0 ? 1u : 0u);
           }
           umma_commit(dp_full);
           if (!mbar_wait(p_ready, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO
-            const uint64_t a = sdesc_sw128(sPSa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO (P^T read MN-major from the P tile)
+            const uint64_t a = sdesc_sw128(sPSa + kk * 2048, 16384, 1024);
             const uint64_t bd = sdesc_sw128(sDOa + kk * 2048, 16384, 1024);
-            umma_bf16_ss(tDV, a, bd, IDESC_KN, (nd > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ss(tDV, a, bd, IDESC_MN, (nd > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(do_empty);
           umma_commit(dv_done);
         }
         if (t + 1 < T) {  // the next tile's scores as early as possible
           if (!mbar_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, fs)) break;
-          if (!mbar_wait(st_free, t & 1, fs)) break;  // S^T(t) consumed
+          if (!mbar_wait(st_free, t & 1, fs)) break;  // S(t) consumed
           tc_fence_after();
           issue_qk((t + 1) & 1);
         }
@@ -268,16 +270,16 @@ __global__ void __launch_bounds__(320, 1)
           if (!mbar_wait(ds_ready, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q
-            const uint64_t a = sdesc_sw128(sPSa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q (dS^T read MN-major from the dS tile)
+            const uint64_t a = sdesc_sw128(sPSa + kk * 2048, 16384, 1024);
             const uint64_t bd = sdesc_sw128(sQs + kk * 2048, 16384, 1024);
-            umma_bf16_ss(tDK, a, bd, IDESC_KN, (nd > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ss(tDK, a, bd, IDESC_MN, (nd > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K (dS read MN-major from the dS^T tile)
-            const uint64_t a = sdesc_sw128(sPSa + kk * 2048, 16384, 1024);
+          for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K
+            const uint64_t a = sdesc_sw128(sPSa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(sKa + kk * 2048, 16384, 1024);
-            umma_bf16_ss(tDP, a, bd, IDESC_DQ, kk > 0 ? 1u : 0u);
+            umma_bf16_ss(tDP, a, bd, IDESC_KN, kk > 0 ? 1u : 0u);
           }
           umma_commit(dq_full);
           umma_commit(ps_free);
@@ -343,9 +345,12 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ compute warpgroup
+    // Thread tid owns query row tid of the current tile (TMEM lane tid of S and
+    // dP): its LSE, gate threshold and D are scalars. The loops over 64-column
+    // halves stay rolled: one warp per SM sub-partition runs this code, and
+    // straight-line code beyond the instruction cache starves it.
     const int tid = threadIdx.x;
-    const int kj = k0 + tid;  // my key
-    const int ki = tid / BK;  // my key block inside the CTA
+    const int qi = tid / BQ;  // my query block inside the tile
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t sPSa = smem_u32(sPS);
     const float sl2 = p.scale_log2;
@@ -357,61 +362,58 @@ __global__ void __launch_bounds__(320, 1)
       const int st = t & 1;
       const int hq = hkv * p.G + t / nqs;
       const int qs = ks + t % nqs;
-      const int i0 = qs * 128;
-      const bool diag = qs == ks;
-      const uint32_t vec_s = smem_u32(sVec + st * 384);  // LSE2 | gate threshold | D, 128 each
+      const bool diag = qs == ks;  // then key column c is live for my row iff c <= tid
+      const float* vec = sVec + st * 384;  // LSE2 | gate threshold | D, 128 each
       const bool ok = mbar_wait_warp(s_full, t & 1, fs);
       local_abort |= !ok;
       tc_fence_after();
-      uint32_t kbits = 0;
+      uint32_t kbits = 0;  // bit kx: my row passes the gate inside key block kx
       if (kGate) {
-        bool hit[QPB];
-#pragma unroll
-        for (int qi = 0; qi < QPB; ++qi) hit[qi] = false;
-#pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {  // S^T row in halves: two loads in flight, one wait
+        const float thr = vec[128 + tid];
+#pragma unroll 1
+        for (int hlf = 0; hlf < 2; ++hlf) {
           uint32_t sh[64];
           tmem_ld32_at(tS + lane_base + hlf * 64, sh);
           tmem_ld32_at(tS + lane_base + hlf * 64 + 32, sh + 32);
           tmem_ld_wait();
-          if (ok) {
+          float m8[8];
 #pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4) {
-              const float4 th = ld_shared_f4(vec_s + 4 * (128 + hlf * 64 + j4 * 4));
-              const float tv[4] = {th.x, th.y, th.z, th.w};
+          for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
+          if (!diag) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int il = hlf * 64 + j4 * 4 + e;
-                const bool live = !diag || (i0 + il >= kj);
-                hit[il / BQ] |= live && (__uint_as_float(sh[j4 * 4 + e]) * sl2 >= tv[e]);
-              }
-            }
+            for (int c = 0; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c]));
+          } else {
+            const int lim = tid - hlf * 64;  // live columns of this half: c <= lim
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], c <= lim ? __uint_as_float(sh[c]) : -INFINITY);
           }
+          const float m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          // max_c(s_c) * sl2 == max_c(s_c * sl2): rounding is monotone
+          if (ok && m * sl2 >= thr) kbits |= 1u << ((hlf * 64) / BK);
         }
-#pragma unroll
-        for (int qi = 0; qi < QPB; ++qi) kbits |= hit[qi] ? (1u << qi) : 0u;
       } else {
 #pragma unroll
-        for (int qi = 0; qi < QPB; ++qi) {
-          const int qb = qs * QPB + qi, kb = ks * KPB + ki;
-          if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) kbits |= 1u << qi;
+        for (int kx = 0; kx < KPB; ++kx) {
+          const int qb = qs * QPB + qi, kb = ks * KPB + kx;
+          if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) kbits |= 1u << kx;
         }
       }
       uint32_t wv = 0;
 #pragma unroll
-      for (int qi = 0; qi < QPB; ++qi) wv |= (__ballot_sync(0xffffffffu, (kbits >> qi) & 1u) ? 1u : 0u) << qi;
+      for (int kx = 0; kx < KPB; ++kx) wv |= (__ballot_sync(0xffffffffu, (kbits >> kx) & 1u) ? 1u : 0u) << kx;
       if (lane == 0) vote[(t & 1) * 4 + warp] = wv | (local_abort ? 8u : 0u);
       named_bar_sync(1, 128);
-      uint32_t kept = 0;  // bit (qi * 2 + ki): sub-tile kept
+      uint32_t kept = 0;  // bit (qi * 2 + kx): sub-tile kept
       bool any_abort = false;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const uint32_t vw = vote[(t & 1) * 4 + w];
         any_abort |= (vw & 8u) != 0;
-        const int kw = (w * 32) / BK;
+        const int qw = (w * 32) / BQ;
 #pragma unroll
-        for (int qi = 0; qi < QPB; ++qi)
-          if ((vw >> qi) & 1u) kept |= 1u << (qi * 2 + kw);
+        for (int kx = 0; kx < KPB; ++kx)
+          if ((vw >> kx) & 1u) kept |= 1u << (qw * 2 + kx);
       }
       if (tid == 0) {
         *dec_flags = kept | (kept ? kBwdAny : 0u) | (any_abort ? kBwdAbort : 0u);
@@ -423,11 +425,11 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (tid == 0) {
         int cnt = 0;
-        for (int qi = 0; qi < QPB; ++qi)
+        for (int qx = 0; qx < QPB; ++qx)
           for (int kx = 0; kx < KPB; ++kx) {
-            const int qb = qs * QPB + qi, kb = ks * KPB + kx;
+            const int qb = qs * QPB + qx, kb = ks * KPB + kx;
             if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) {
-              const int kp = (kept >> (qi * 2 + kx)) & 1u;
+              const int kp = (kept >> (qx * 2 + kx)) & 1u;
               if (p.keep_map) p.keep_map[(static_cast<size_t>(b * p.Hq + hq) * p.nq + qb) * p.nk + kb] = kp;
               cnt += kp;
             }
@@ -439,68 +441,63 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive(st_free);
         continue;
       }
-      // ---- kept: P^T row of my key, zero outside kept sub-tiles / live entries
+      // ---- kept: P row of my query, zero outside kept sub-tiles / live entries
       if (nd >= 1) local_abort |= !mbar_wait_warp(ps_free, (nd - 1) & 1, fs);
-      uint32_t qmask = 0;  // query blocks whose sub-tile with my key block is kept
-#pragma unroll
-      for (int qi = 0; qi < QPB; ++qi) qmask |= ((kept >> (qi * 2 + ki)) & 1u) << qi;
-#pragma unroll
+      const float lse2 = vec[tid];  // +inf for rows at or past L: their P is 0
+      const uint32_t kmask = (kept >> (qi * 2)) & 3u;  // key blocks kept for my query block
+#pragma unroll 1
       for (int hlf = 0; hlf < 2; ++hlf) {
         uint32_t sh[64];
         tmem_ld32_at(tS + lane_base + hlf * 64, sh);
         tmem_ld32_at(tS + lane_base + hlf * 64 + 32, sh + 32);
         tmem_ld_wait();
+        const bool on = (kmask >> ((hlf * 64) / BK)) & 1u;  // warp-uniform
+        const int lim = diag ? tid - hlf * 64 : 63;  // live columns: c <= lim
+        uint32_t pk[32];
+        if (on && !diag) {
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          const int ch = hlf * 2 + c2;
-          uint32_t pk[16];
+          for (int jj = 0; jj < 32; ++jj)
+            pk[jj] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sh[2 * jj]), sl2, -lse2)),
+                                 ex2_approx(fmaf(__uint_as_float(sh[2 * jj + 1]), sl2, -lse2)));
+        } else {
+          // dead entries go through ex2 as -inf (-> 0): no branch around the inline asm
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int il = ch * 32 + 2 * jj;
-            const float2 lv = ld_shared_f2(vec_s + 4 * il);
-            const bool l0 = ((qmask >> (il / BQ)) & 1u) && (!diag || i0 + il >= kj);
-            const bool l1 = ((qmask >> ((il + 1) / BQ)) & 1u) && (!diag || i0 + il + 1 >= kj);
-            // dead entries go through ex2 as -inf (-> 0): no branch around the inline asm
-            const float p0 = ex2_approx(l0 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -lv.x) : -INFINITY);
-            const float p1 = ex2_approx(l1 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj + 1]), sl2, -lv.y) : -INFINITY);
-            pk[jj] = pack_bf16x2(p0, p1);
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int col = ch * 32 + c * 8;
-            st_shared_v4(sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pk[4 * c],
-                         pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int jj = 0; jj < 32; ++jj) {
+            const bool l0 = on && 2 * jj <= lim, l1 = on && 2 * jj + 1 <= lim;
+            pk[jj] = pack_bf16x2(ex2_approx(l0 ? fmaf(__uint_as_float(sh[2 * jj]), sl2, -lse2) : -INFINITY),
+                                 ex2_approx(l1 ? fmaf(__uint_as_float(sh[2 * jj + 1]), sl2, -lse2) : -INFINITY));
           }
         }
+        const uint32_t rowa = sPSa + hlf * 16384;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(rowa + sw128_offset(tid, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_ready);
       mbar_arrive(st_free);
-      // ---- dS^T = P^T * (dP^T - D), written over P^T once the dV MMA has read it
+      // ---- dS = P * (dP - D), written over P once the dV MMA has read it
+      const float dsub = vec[256 + tid];
       local_abort |= !mbar_wait_warp(dp_full, nd & 1, fs);
       local_abort |= !mbar_wait_warp(dv_done, nd & 1, fs);
       tc_fence_after();
-#pragma unroll
+#pragma unroll 1
       for (int hlf = 0; hlf < 2; ++hlf) {
         uint32_t dh[64];
         tmem_ld32_at(tDP + lane_base + hlf * 64, dh);
         tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, dh + 32);
         tmem_ld_wait();
+        const uint32_t rowa = sPSa + hlf * 16384;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const int col = hlf * 64 + c * 8;
-          const uint32_t addr = sPSa + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3);
+          const uint32_t addr = rowa + sw128_offset(tid, c);
           uint32_t pp[4], ds[4];
           ld_shared_v4(addr, pp[0], pp[1], pp[2], pp[3]);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int il = col + 2 * e;
-            const float2 dv2 = ld_shared_f2(vec_s + 4 * (256 + il));
-            const float d0 = __uint_as_float(dh[c * 8 + 2 * e]) - dv2.x;
-            const float d1 = __uint_as_float(dh[c * 8 + 2 * e + 1]) - dv2.y;
-            ds[e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * d0, bf16hi_to_f32(pp[e]) * d1);
-          }
+          for (int e = 0; e < 4; ++e)
+            ds[e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * (__uint_as_float(dh[c * 8 + 2 * e]) - dsub),
+                                bf16hi_to_f32(pp[e]) * (__uint_as_float(dh[c * 8 + 2 * e + 1]) - dsub));
           st_shared_v4(addr, ds[0], ds[1], ds[2], ds[3]);
         }
       }
