@@ -134,7 +134,7 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   auto kern = mala::mala_bwd_kernel<D, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.n_super) * p.B * p.Hkv;
-  kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  kern<<<grid, 448, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 

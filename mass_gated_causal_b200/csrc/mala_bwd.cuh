@@ -62,22 +62,22 @@ struct BwdLayout {
   static constexpr int OFF_Q = OFF_V + T_BYTES;  // 2 stages
   static constexpr int OFF_DO = OFF_Q + 2 * T_BYTES;
   static constexpr int OFF_PS = OFF_DO + T_BYTES;
-  static constexpr int STG_WARP = 32 * 32 * 4;  // dQ staging: [32 rows x 32] fp32 per drain warp
+  static constexpr int STG_BUF = 32 * 32 * 4;   // dQ staging block: [32 rows x 32] fp32
+  static constexpr int STG_WARP = 2 * STG_BUF;  // two blocks per drain warp
   static constexpr int OFF_STG = OFF_PS + PS_BYTES;  // 1024-aligned (128-byte swizzle)
-  static constexpr int OFF_VEC = OFF_STG + 4 * STG_WARP;  // [2 stages][LSE2, T, D][128] fp32
-  static constexpr int OFF_BAR = OFF_VEC + 2 * 3 * 128 * 4;
-  // kv_full, q_full[2], q_empty[2], s_full, st_free, dec, do_full, do_empty,
-  // dp_full, p_ready, dv_done, ds_ready, dq_full, dq_free, ps_free, mma_final, info_full
-  static constexpr int N_BARS = 19;
+  static constexpr int OFF_BAR = OFF_STG + 4 * STG_WARP;
+  // kv_full, q_full[2], q_empty[2], s_full, dec, do_full, do_empty, p_ready,
+  // dv_done, ds_ready, dq_full, dq_free, ps_free, mma_final, info_full
+  static constexpr int N_BARS = 17;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-  static constexpr int BYTES = OFF_MISC + 96;
+  static constexpr int BYTES = OFF_MISC + 128;
   static constexpr int ALLOC_BYTES = BYTES + 1024;
   static constexpr int TMEM_COLS = 512;  // S 128 | dP/dQ 128 | dK D | dV D
   static_assert(ALLOC_BYTES <= 232448, "backward shared memory exceeds the per-CTA limit");
 };
 
 template <int D, int BK, bool kGate>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     mala_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(320, 1)
   constexpr uint32_t IDESC_KN = idesc_bf16(128, D, false, true);  // A K-major, B MN-major
   constexpr uint32_t IDESC_MN = idesc_bf16(128, D, true, true);   // A, B MN-major
   constexpr int TB = Lay::T_BYTES;
+  constexpr uint32_t kNegInfBits = 0xff800000u;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -96,32 +97,29 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sQ = smem + Lay::OFF_Q;
   uint8_t* sDO = smem + Lay::OFF_DO;
   uint8_t* sPS = smem + Lay::OFF_PS;
-  float* sVec = reinterpret_cast<float*>(smem + Lay::OFF_VEC);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;   // [2]
   uint64_t* q_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;
-  uint64_t* st_free = bars + 6;
-  uint64_t* dec_bar = bars + 7;
-  uint64_t* do_full = bars + 8;
-  uint64_t* do_empty = bars + 9;
-  uint64_t* dp_full = bars + 10;
-  uint64_t* p_ready = bars + 11;
-  uint64_t* dv_done = bars + 12;
-  uint64_t* ds_ready = bars + 13;
-  uint64_t* dq_full = bars + 14;
-  uint64_t* dq_free = bars + 15;
-  uint64_t* ps_free = bars + 16;
-  uint64_t* mma_final = bars + 17;
-  uint64_t* info_full = bars + 18;
+  uint64_t* dec_bar = bars + 6;  // also tells the MMA issuer that S(t) is out of TMEM
+  uint64_t* do_full = bars + 7;
+  uint64_t* do_empty = bars + 8;
+  uint64_t* p_ready = bars + 9;
+  uint64_t* dv_done = bars + 10;  // dP(t) was issued before dV(t): its completion too
+  uint64_t* ds_ready = bars + 11;
+  uint64_t* dq_full = bars + 12;
+  uint64_t* dq_free = bars + 13;
+  uint64_t* ps_free = bars + 14;
+  uint64_t* mma_final = bars + 15;
+  uint64_t* info_full = bars + 16;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   uint32_t* tmem_slot = misc + 0;
   int* abort_flag = reinterpret_cast<int*>(misc + 1);
   uint32_t* dec_flags = misc + 2;
-  uint32_t* vote = misc + 4;    // [2][4]
-  uint32_t* evote = misc + 12;  // [4]
-  int* info = reinterpret_cast<int*>(misc + 16);  // {hq, i0} of the kept tile the drain warpgroup handles next
+  uint32_t* vote = misc + 4;    // [2][8]
+  uint32_t* evote = misc + 20;  // [8]
+  int* info = reinterpret_cast<int*>(misc + 28);  // {hq, i0, TMEM region} of the next kept tile to drain
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -136,18 +134,16 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 33);  // expect_tx arrival + 32 vector-writing lanes
+      mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(st_free, 128);
     mbar_init(dec_bar, 1);
     mbar_init(do_full, 1);
     mbar_init(do_empty, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(p_ready, 128);
+    mbar_init(p_ready, 256);
     mbar_init(dv_done, 1);
-    mbar_init(ds_ready, 128);
+    mbar_init(ds_ready, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     mbar_init(ps_free, 1);
@@ -156,7 +152,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, Lay::TMEM_COLS);
     tmem_relinquish();
   }
@@ -165,9 +161,11 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   const FailState fs{abort_flag, p.status};
-  const uint32_t tS = tmem, tDP = tmem + 128, tDK = tmem + 256, tDV = tmem + 256 + D;
+  // TMEM: two 128-column regions taken by tiles in turn (tile t uses region
+  // t & 1 for S, then dP, then dQ), then dK and dV.
+  const uint32_t tDK = tmem + 256, tDV = tmem + 256 + D;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * TB);
@@ -176,7 +174,7 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_4d(&tm_v, kv_full, sV + h * 16384, h * 64, hkv, k0, b);
       }
     }
-    int issued = 0;
+    int issued_q = 0, issued_do = 0;
     for (int t = 0; t < T; ++t) {
       const int st = t & 1;
       if (t >= 2 && !mbar_wait_warp(&q_empty[st], ((t >> 1) - 1) & 1, fs)) break;
@@ -186,234 +184,259 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive_expect_tx(&q_full[st], TB);
         for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_q, &q_full[st], sQ + st * TB + h * 16384, h * 64, hq, i0, b);
       }
-      float* vec = sVec + st * 384;
-      const size_t rowbase = static_cast<size_t>(b * p.Hq + hq) * p.L;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = lane * 4 + e;
-        const int i = i0 + r;
-        const bool ok = i < p.L;
-        const float lse2 = ok ? p.lse[rowbase + i] * 1.4426950408889634f : INFINITY;
-        vec[r] = lse2;
-        vec[128 + r] = kGate ? lse2 + p.log2_tau - lg2_approx(static_cast<float>(i + 1)) : 0.f;
-        vec[256 + r] = ok ? p.dvec[rowbase + i] : 0.f;
+      issued_q = t + 1;
+      // dO of the same tile, before the gate has decided: the buffer is free as
+      // soon as the previous tile's dP and dV have read it, and nearly every
+      // tile is kept
+      if (t >= 1 && !mbar_wait_warp(do_empty, (t - 1) & 1, fs)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(do_full, TB);
+        for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, i0, b);
       }
-      mbar_arrive(&q_full[st]);
-      issued = t + 1;
+      issued_do = t + 1;
     }
     if (lane == 0) {
       mbar_wait_drain(kv_full, 0);
-      for (int t = max(0, issued - 2); t < issued; ++t) mbar_wait_drain(&q_full[t & 1], (t >> 1) & 1);
+      for (int t = max(0, issued_q - 2); t < issued_q; ++t) mbar_wait_drain(&q_full[t & 1], (t >> 1) & 1);
+      if (issued_do >= 1) mbar_wait_drain(do_full, (issued_do - 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
-      const uint32_t sPSa = smem_u32(sPS);
+      // operand descriptors, built once: K-major (k-steps inside 64-column
+      // atoms) and MN-major (k-steps of 16 rows) views of each tile
+      const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024), dKm = sdesc_sw128(smem_u32(sK), 16384, 1024);
+      const uint64_t dVk = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024), dQm = sdesc_sw128(smem_u32(sQ), 16384, 1024);
+      const uint64_t dOk = sdesc_sw128(smem_u32(sDO), 16, 1024), dOm = sdesc_sw128(smem_u32(sDO), 16384, 1024);
+      const uint64_t dPk = sdesc_sw128(smem_u32(sPS), 16, 1024), dPm = sdesc_sw128(smem_u32(sPS), 16384, 1024);
       int nd = 0;
-      auto issue_qk = [&](int st) {  // S = Q K^T
+      int reg_kept0 = -1, reg_kept1 = -1;  // kept-tile index whose dQ still occupies region 0 / 1
+      int dq_seen = -1;                    // highest kept-tile index whose dQ is known drained
+      // S(t) = Q K^T into region t & 1, once Q(t) has landed and the dQ that
+      // last used the region has been drained (one wait for both)
+      auto issue_qk = [&](int t) -> bool {
+        const int r = t & 1;
+        const int pend = r ? reg_kept1 : reg_kept0;
+        if (pend >= 0) {
+          if (!mbar_wait2(&q_full[t & 1], (t >> 1) & 1, dq_free, pend & 1, fs)) return false;
+          dq_seen = max(dq_seen, pend);
+          if (r) reg_kept1 = -1; else reg_kept0 = -1;
+        } else if (!mbar_wait(&q_full[t & 1], (t >> 1) & 1, fs)) {
+          return false;
+        }
+        tc_fence_after();
+        const uint64_t qa = sdesc_add(dQk, (t & 1) * TB);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(tS, sdesc_sw128(sQa + st * TB + off, 16, 1024), sdesc_sw128(sKa + off, 16, 1024), IDESC_S,
-                       kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + r * 128, sdesc_add(qa, off), sdesc_add(dKk, off), IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full);
+        return true;
       };
-      bool ok = mbar_wait(kv_full, 0, fs) && mbar_wait(&q_full[0], 0, fs);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-      }
+      bool ok = mbar_wait(kv_full, 0, fs);
+      if (ok) ok = issue_qk(0);
       for (int t = 0; ok && t < T; ++t) {
         const int st = t & 1;
         const int hq = hkv * p.G + t / nqs;
         const int i0 = (ks + t % nqs) * 128;
-        const uint32_t sQs = sQa + st * TB;
-        if (!mbar_wait(dec_bar, t & 1, fs)) break;
+        const uint32_t tR = tmem + (t & 1) * 128;
+        // the gate's decision (the compute warps have read S(t) out of the
+        // region before voting) and dO(t), loaded ahead: one wait for both
+        if (!mbar_wait2(dec_bar, t & 1, do_full, t & 1, fs)) break;
         const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(dec_flags);
         if (dec & kBwdAbort) break;
         const bool keep = (dec & kBwdAny) != 0;
         if (keep) {
-          if (nd >= 1 && !mbar_wait(do_empty, (nd - 1) & 1, fs)) break;
-          mbar_arrive_expect_tx(do_full, TB);
-          for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, i0, b);
-          if (nd >= 1 && !mbar_wait(dq_free, (nd - 1) & 1, fs)) break;  // dQ(nd-1) drained from the dP columns
-          if (!mbar_wait(do_full, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {  // dP = dO V^T
+          for (int kk = 0; kk < D / 16; ++kk) {  // dP = dO V^T, over S in the same region
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16_ss(tDP, sdesc_sw128(sDOa + off, 16, 1024), sdesc_sw128(sVa + off, 16, 1024), IDESC_S,
-                         kk > 0 ? 1u : 0u);
+            umma_bf16_ss(tR, sdesc_add(dOk, off), sdesc_add(dVk, off), IDESC_S, kk > 0 ? 1u : 0u);
           }
-          umma_commit(dp_full);
           if (!mbar_wait(p_ready, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO (P^T read MN-major from the P tile)
-            const uint64_t a = sdesc_sw128(sPSa + kk * 2048, 16384, 1024);
-            const uint64_t bd = sdesc_sw128(sDOa + kk * 2048, 16384, 1024);
-            umma_bf16_ss(tDV, a, bd, IDESC_MN, (nd > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ss(tDV, sdesc_add(dPm, kk * 2048), sdesc_add(dOm, kk * 2048), IDESC_MN,
+                         (nd > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(do_empty);
+          umma_commit(do_empty);  // dO(t): read by dP and dV
           umma_commit(dv_done);
+        } else {
+          mbar_arrive(do_empty);  // dO(t) is not needed
         }
-        if (t + 1 < T) {  // the next tile's scores as early as possible
-          if (!mbar_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, fs)) break;
-          if (!mbar_wait(st_free, t & 1, fs)) break;  // S(t) consumed
-          tc_fence_after();
-          issue_qk((t + 1) & 1);
-        }
+        if (t + 1 < T && !issue_qk(t + 1)) break;  // the next tile's scores, into the other region
         if (keep) {
           if (!mbar_wait(ds_ready, nd & 1, fs)) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // dK += dS^T Q (dS^T read MN-major from the dS tile)
-            const uint64_t a = sdesc_sw128(sPSa + kk * 2048, 16384, 1024);
-            const uint64_t bd = sdesc_sw128(sQs + kk * 2048, 16384, 1024);
-            umma_bf16_ss(tDK, a, bd, IDESC_MN, (nd > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ss(tDK, sdesc_add(dPm, kk * 2048), sdesc_add(dQm, st * TB + kk * 2048), IDESC_MN,
+                         (nd > 0 || kk > 0) ? 1u : 0u);
+          }
+          // the drain warps have taken the previous kept tile (info slot free)
+          if (nd >= 1 && dq_seen < nd - 1) {
+            if (!mbar_wait(dq_free, (nd - 1) & 1, fs)) break;
+            dq_seen = nd - 1;
           }
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K
-            const uint64_t a = sdesc_sw128(sPSa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sKa + kk * 2048, 16384, 1024);
-            umma_bf16_ss(tDP, a, bd, IDESC_KN, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {  // dQ = dS K, over dP in the same region
+            umma_bf16_ss(tR, sdesc_add(dPk, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(dKm, kk * 2048), IDESC_KN,
+                         kk > 0 ? 1u : 0u);
           }
           umma_commit(dq_full);
           umma_commit(ps_free);
-          info[0] = hq;  // the drain warpgroup finished dQ(nd-1) before dP(nd) was issued
+          info[0] = hq;
           info[1] = i0;
+          info[2] = t & 1;
           mbar_arrive(info_full);
+          if (t & 1) reg_kept1 = nd; else reg_kept0 = nd;
           ++nd;
         }
         umma_commit(&q_empty[st]);  // Q(t): QK(t) and dK(t) issued
       }
-      // tell the drain warpgroup there is nothing more, once it has taken the last tile
+      // tell the drain warps there is nothing more, once they have taken the last tile
       if (nd >= 1) mbar_wait(dq_free, (nd - 1) & 1, fs);
       info[0] = -1;
       mbar_arrive(info_full);
       umma_commit(mma_final);
-      if (nd >= 1) mbar_wait_drain(do_full, (nd - 1) & 1);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ dQ drain warpgroup
-    // Warp w owns query rows [32w, 32w+32) of each kept tile (TMEM lanes of the
-    // dQ accumulator). It reads its rows out of TMEM, hands the columns back to
-    // the MMA issuer, and adds them to the fp32 workspace 32 columns at a time:
-    // a swizzled [32 x 32] fp32 block in shared memory, reduced into global
-    // memory by one TMA add (whole 128-byte lines, element-wise atomic adds).
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ drain warps
+    // Warp 8 + w owns query rows [32w, 32w+32) of each kept tile (TMEM lanes of
+    // the dQ accumulator). It reads its rows out of TMEM, hands the region back
+    // to the MMA issuer, and adds them to the fp32 workspace 32 columns at a
+    // time: a swizzled [32 x 32] fp32 block in shared memory, reduced into
+    // global memory by one TMA add (whole 128-byte lines, element-wise atomic;
+    // per-thread atomics from registers are several times slower at the L2).
     const int wq = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint8_t* stg = smem + Lay::OFF_STG + wq * Lay::STG_WARP;
-    const uint32_t stg_s = smem_u32(stg);
     for (int n = 0;; ++n) {
       if (!mbar_wait_warp(info_full, n & 1, fs)) break;
       const int hq = *reinterpret_cast<volatile int*>(&info[0]);
       const int i0 = *reinterpret_cast<volatile int*>(&info[1]);
+      const int reg = *reinterpret_cast<volatile int*>(&info[2]);
       if (hq < 0) break;
       if (!mbar_wait_warp(dq_full, n & 1, fs)) break;
       tc_fence_after();
-      uint32_t qh[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32_at(tDP + lane_base + c * 32, qh + c * 32);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(dq_free);
       const int row0 = i0 + wq * 32;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        if (lane == 0) bulk_wait_read0();  // the previous block has left the staging buffer
-        __syncwarp();
+      for (int hb = 0; hb < D / 64; ++hb) {  // 64 columns at a time
+        uint32_t qh[64];
+        tmem_ld32_at(tmem + reg * 128 + lane_base + hb * 64, qh);
+        tmem_ld32_at(tmem + reg * 128 + lane_base + hb * 64 + 32, qh + 32);
+        tmem_ld_wait();
+        if (hb == D / 64 - 1) {  // the region goes back to the MMA issuer
+          tc_fence_before();
+          mbar_arrive(dq_free);
+        }
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(stg_s + sw128_offset(lane, j), __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j])),
-                       __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j + 1])),
-                       __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j + 2])),
-                       __float_as_uint(p.scale * __uint_as_float(qh[c * 32 + 4 * j + 3])));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && row0 < p.L) {  // rows at or past L are clipped by the tensor map
-          tma_reduce_add_4d(&tm_dq, stg, c * 32, hq, row0, b);
-          bulk_commit();
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int c = hb * 2 + c2;
+          uint8_t* buf = stg + (c & 1) * Lay::STG_BUF;
+          const uint32_t buf_s = smem_u32(buf);
+          if (lane == 0) bulk_wait_read1();  // the block two steps back has left this buffer
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(buf_s + sw128_offset(lane, j),
+                         __float_as_uint(p.scale * __uint_as_float(qh[c2 * 32 + 4 * j])),
+                         __float_as_uint(p.scale * __uint_as_float(qh[c2 * 32 + 4 * j + 1])),
+                         __float_as_uint(p.scale * __uint_as_float(qh[c2 * 32 + 4 * j + 2])),
+                         __float_as_uint(p.scale * __uint_as_float(qh[c2 * 32 + 4 * j + 3])));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < p.L) tma_reduce_add_4d(&tm_dq, buf, c * 32, hq, row0, b);  // rows past L are clipped
+            bulk_commit();  // one group per block, empty when skipped, so the counting above holds
+          }
         }
       }
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ compute warpgroup
-    // Thread tid owns query row tid of the current tile (TMEM lane tid of S and
-    // dP): its LSE, gate threshold and D are scalars. The loops over 64-column
-    // halves stay rolled: one warp per SM sub-partition runs this code, and
-    // straight-line code beyond the instruction cache starves it.
+    // ------------------------------------------------------------ compute warps
+    // Thread tid owns query row (tid % 128) of the current tile, key columns
+    // [64h, 64h + 64) with h = tid / 128 (TMEM lane row, 64 columns of S and dP
+    // in the tile's region): its LSE, gate threshold and D are scalars. At the
+    // end, thread tid writes key row (tid % 128), half h of the columns of dK
+    // and dV.
     const int tid = threadIdx.x;
-    const int qi = tid / BQ;  // my query block inside the tile
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t sPSa = smem_u32(sPS);
+    const int row = tid & 127;
+    const int kh = tid >> 7;
+    const int qi = row / BQ;        // my query block inside the tile
+    const int kx = (kh * 64) / BK;  // my key block inside the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t psa = smem_u32(sPS) + kh * 16384;  // my 64-column atom of the P / dS tile
     const float sl2 = p.scale_log2;
     int nd = 0;
     bool local_abort = false, all_abort = false;
-    uint32_t r[32];
+    // LSE and D of my row, loaded one tile ahead (rows at or past L: LSE +inf, D 0)
+    auto row_lse = [&](int t) {
+      const int i = (ks + t % nqs) * 128 + row;
+      return i < p.L ? __ldg(p.lse + static_cast<size_t>(b * p.Hq + hkv * p.G + t / nqs) * p.L + i) : INFINITY;
+    };
+    auto row_d = [&](int t) {
+      const int i = (ks + t % nqs) * 128 + row;
+      return i < p.L ? __ldg(p.dvec + static_cast<size_t>(b * p.Hq + hkv * p.G + t / nqs) * p.L + i) : 0.f;
+    };
+    float lse_next = row_lse(0), d_next = row_d(0);
 
     for (int t = 0; t < T; ++t) {
-      const int st = t & 1;
       const int hq = hkv * p.G + t / nqs;
       const int qs = ks + t % nqs;
-      const bool diag = qs == ks;  // then key column c is live for my row iff c <= tid
-      const float* vec = sVec + st * 384;  // LSE2 | gate threshold | D, 128 each
+      const bool diag = qs == ks;  // then key column c is live for my row iff c <= row
+      const float lse2_row = lse_next * 1.4426950408889634f, d_row = d_next;
+      if (t + 1 < T) {
+        lse_next = row_lse(t + 1);
+        d_next = row_d(t + 1);
+      }
+      const uint32_t tR = tmem + (t & 1) * 128 + kh * 64 + lane_base;
       const bool ok = mbar_wait_warp(s_full, t & 1, fs);
       local_abort |= !ok;
       tc_fence_after();
-      uint32_t kbits = 0;  // bit kx: my row passes the gate inside key block kx
-      if (kGate) {
-        const float thr = vec[128 + tid];
-#pragma unroll 1
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          uint32_t sh[64];
-          tmem_ld32_at(tS + lane_base + hlf * 64, sh);
-          tmem_ld32_at(tS + lane_base + hlf * 64 + 32, sh + 32);
-          tmem_ld_wait();
-          float m8[8];
+      uint32_t sh[64];
+      tmem_ld32_at(tR, sh);
+      tmem_ld32_at(tR + 32, sh + 32);
+      tmem_ld_wait();
+      tc_fence_before();  // S(t) is in registers: after the vote the MMA may write dP over it
+      if (diag) {
+        const int lim = row - kh * 64;  // live columns: c <= lim
 #pragma unroll
-          for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
-          if (!diag) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c]));
-          } else {
-            const int lim = tid - hlf * 64;  // live columns of this half: c <= lim
-#pragma unroll
-            for (int c = 0; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], c <= lim ? __uint_as_float(sh[c]) : -INFINITY);
-          }
-          const float m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-          // max_c(s_c) * sl2 == max_c(s_c * sl2): rounding is monotone
-          if (ok && m * sl2 >= thr) kbits |= 1u << ((hlf * 64) / BK);
-        }
-      } else {
-#pragma unroll
-        for (int kx = 0; kx < KPB; ++kx) {
-          const int qb = qs * QPB + qi, kb = ks * KPB + kx;
-          if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) kbits |= 1u << kx;
-        }
+        for (int c = 0; c < 64; ++c) sh[c] = c <= lim ? sh[c] : kNegInfBits;
       }
-      uint32_t wv = 0;
+      bool hit;
+      if (kGate) {
+        float m8[8];
 #pragma unroll
-      for (int kx = 0; kx < KPB; ++kx) wv |= (__ballot_sync(0xffffffffu, (kbits >> kx) & 1u) ? 1u : 0u) << kx;
-      if (lane == 0) vote[(t & 1) * 4 + warp] = wv | (local_abort ? 8u : 0u);
-      named_bar_sync(1, 128);
+        for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sh[e]);
+#pragma unroll
+        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c]));
+        const float m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        // max_c(s_c) * sl2 == max_c(s_c * sl2): rounding is monotone
+        const float thr = lse2_row + p.log2_tau - lg2_approx(static_cast<float>(qs * 128 + row + 1));
+        hit = ok && m * sl2 >= thr;
+      } else {
+        const int qb = qs * QPB + qi, kb = ks * KPB + kx;
+        hit = qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, hit);
+      if (lane == 0) vote[(t & 1) * 8 + warp] = (bal ? 1u : 0u) | (local_abort ? 8u : 0u);
+      named_bar_sync(1, 256);
       uint32_t kept = 0;  // bit (qi * 2 + kx): sub-tile kept
       bool any_abort = false;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t vw = vote[(t & 1) * 4 + w];
+      for (int w = 0; w < 8; ++w) {
+        const uint32_t vw = vote[(t & 1) * 8 + w];
         any_abort |= (vw & 8u) != 0;
-        const int qw = (w * 32) / BQ;
-#pragma unroll
-        for (int kx = 0; kx < KPB; ++kx)
-          if ((vw >> kx) & 1u) kept |= 1u << (qw * 2 + kx);
+        if (vw & 1u) kept |= 1u << ((((w & 3) * 32) / BQ) * 2 + ((w >> 2) * 64) / BK);
       }
       if (tid == 0) {
         *dec_flags = kept | (kept ? kBwdAny : 0u) | (any_abort ? kBwdAbort : 0u);
@@ -426,80 +449,48 @@ __global__ void __launch_bounds__(320, 1)
       if (tid == 0) {
         int cnt = 0;
         for (int qx = 0; qx < QPB; ++qx)
-          for (int kx = 0; kx < KPB; ++kx) {
-            const int qb = qs * QPB + qx, kb = ks * KPB + kx;
+          for (int kz = 0; kz < KPB; ++kz) {
+            const int qb = qs * QPB + qx, kb = ks * KPB + kz;
             if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) {
-              const int kp = (kept >> (qx * 2 + kx)) & 1u;
+              const int kp = (kept >> (qx * 2 + kz)) & 1u;
               if (p.keep_map) p.keep_map[(static_cast<size_t>(b * p.Hq + hq) * p.nq + qb) * p.nk + kb] = kp;
               cnt += kp;
             }
           }
         if (cnt) atomicAdd(&p.kept_tiles[b * p.Hq + hq], cnt);
       }
-      if (!kept) {
-        tc_fence_before();
-        mbar_arrive(st_free);
-        continue;
-      }
-      // ---- kept: P row of my query, zero outside kept sub-tiles / live entries
-      if (nd >= 1) local_abort |= !mbar_wait_warp(ps_free, (nd - 1) & 1, fs);
-      const float lse2 = vec[tid];  // +inf for rows at or past L: their P is 0
-      const uint32_t kmask = (kept >> (qi * 2)) & 3u;  // key blocks kept for my query block
-#pragma unroll 1
-      for (int hlf = 0; hlf < 2; ++hlf) {
-        uint32_t sh[64];
-        tmem_ld32_at(tS + lane_base + hlf * 64, sh);
-        tmem_ld32_at(tS + lane_base + hlf * 64 + 32, sh + 32);
-        tmem_ld_wait();
-        const bool on = (kmask >> ((hlf * 64) / BK)) & 1u;  // warp-uniform
-        const int lim = diag ? tid - hlf * 64 : 63;  // live columns: c <= lim
-        uint32_t pk[32];
-        if (on && !diag) {
+      if (!kept) continue;
+      // ---- kept: P of my row and columns; a sub-tile that is not kept gives 0
+      // (LSE taken as +inf), so do masked entries (-inf scores)
+      const float lse2 = ((kept >> (qi * 2 + kx)) & 1u) ? lse2_row : INFINITY;
+      uint32_t pk[32];
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj)
-            pk[jj] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sh[2 * jj]), sl2, -lse2)),
-                                 ex2_approx(fmaf(__uint_as_float(sh[2 * jj + 1]), sl2, -lse2)));
-        } else {
-          // dead entries go through ex2 as -inf (-> 0): no branch around the inline asm
+      for (int jj = 0; jj < 32; ++jj)
+        pk[jj] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sh[2 * jj]), sl2, -lse2)),
+                             ex2_approx(fmaf(__uint_as_float(sh[2 * jj + 1]), sl2, -lse2)));
+      if (nd >= 1) local_abort |= !mbar_wait_warp(ps_free, (nd - 1) & 1, fs);  // dK, dQ of the last tile done
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const bool l0 = on && 2 * jj <= lim, l1 = on && 2 * jj + 1 <= lim;
-            pk[jj] = pack_bf16x2(ex2_approx(l0 ? fmaf(__uint_as_float(sh[2 * jj]), sl2, -lse2) : -INFINITY),
-                                 ex2_approx(l1 ? fmaf(__uint_as_float(sh[2 * jj + 1]), sl2, -lse2) : -INFINITY));
-          }
-        }
-        const uint32_t rowa = sPSa + hlf * 16384;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(rowa + sw128_offset(tid, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(psa + sw128_offset(row, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       fence_proxy_async_smem();
-      tc_fence_before();
       mbar_arrive(p_ready);
-      mbar_arrive(st_free);
       // ---- dS = P * (dP - D), written over P once the dV MMA has read it
-      const float dsub = vec[256 + tid];
-      local_abort |= !mbar_wait_warp(dp_full, nd & 1, fs);
-      local_abort |= !mbar_wait_warp(dv_done, nd & 1, fs);
+      const float dsub = d_row;
+      local_abort |= !mbar_wait_warp(dv_done, nd & 1, fs);  // dP(t) and dV(t) done
       tc_fence_after();
-#pragma unroll 1
-      for (int hlf = 0; hlf < 2; ++hlf) {
-        uint32_t dh[64];
-        tmem_ld32_at(tDP + lane_base + hlf * 64, dh);
-        tmem_ld32_at(tDP + lane_base + hlf * 64 + 32, dh + 32);
-        tmem_ld_wait();
-        const uint32_t rowa = sPSa + hlf * 16384;
+      uint32_t dh[64];
+      tmem_ld32_at(tR, dh);
+      tmem_ld32_at(tR + 32, dh + 32);
+      tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t addr = rowa + sw128_offset(tid, c);
-          uint32_t pp[4], ds[4];
-          ld_shared_v4(addr, pp[0], pp[1], pp[2], pp[3]);
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t addr = psa + sw128_offset(row, c);
+        uint32_t ds[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            ds[e] = pack_bf16x2(bf16lo_to_f32(pp[e]) * (__uint_as_float(dh[c * 8 + 2 * e]) - dsub),
-                                bf16hi_to_f32(pp[e]) * (__uint_as_float(dh[c * 8 + 2 * e + 1]) - dsub));
-          st_shared_v4(addr, ds[0], ds[1], ds[2], ds[3]);
-        }
+        for (int e = 0; e < 4; ++e)  // P of the same entries, still in registers
+          ds[e] = pack_bf16x2(bf16lo_to_f32(pk[4 * c + e]) * (__uint_as_float(dh[c * 8 + 2 * e]) - dsub),
+                              bf16hi_to_f32(pk[4 * c + e]) * (__uint_as_float(dh[c * 8 + 2 * e + 1]) - dsub));
+        st_shared_v4(addr, ds[0], ds[1], ds[2], ds[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -509,6 +500,8 @@ __global__ void __launch_bounds__(320, 1)
 
     if (!all_abort) {
       // ---------------------------------------------------------- epilogue
+      // dK (times the softmax scale) and dV of key row `row`, column half kh,
+      // staged over the Q ring and stored by TMA.
       const bool okf = mbar_wait_warp(mma_final, 0, fs);
       tc_fence_after();
       const uint32_t sQa = smem_u32(sQ);
@@ -519,7 +512,9 @@ __global__ void __launch_bounds__(320, 1)
           const float mul = which == 0 ? p.scale : 1.f;
           const uint32_t dst = sQa + which * TB;
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
+          for (int cc = 0; cc < D / 64; ++cc) {
+            const int ch = kh * (D / 64) + cc;  // 32-column chunk
+            uint32_t r[32];
             if (nd > 0) {
               tmem_ld32(tsrc + ch * 32, r);
               tmem_ld_wait();
@@ -534,7 +529,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               const int col = ch * 32 + c * 8;
-              st_shared_v4(dst + (col >> 6) * 16384 + sw128_offset(tid, (col & 63) >> 3), pk[4 * c], pk[4 * c + 1],
+              st_shared_v4(dst + (col >> 6) * 16384 + sw128_offset(row, (col & 63) >> 3), pk[4 * c], pk[4 * c + 1],
                            pk[4 * c + 2], pk[4 * c + 3]);
             }
           }
@@ -543,8 +538,11 @@ __global__ void __launch_bounds__(320, 1)
       }
       const unsigned okall = __ballot_sync(0xffffffffu, okf);
       if (lane == 0) evote[warp] = okall == 0xffffffffu ? 1u : 0u;
-      named_bar_sync(1, 128);
-      if (tid == 0 && (evote[0] & evote[1] & evote[2] & evote[3])) {
+      named_bar_sync(1, 256);
+      uint32_t all_ok = 1u;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) all_ok &= evote[w];
+      if (tid == 0 && all_ok) {
         for (int h = 0; h < D / 64; ++h) {
           tma_store_4d(&tm_dk, sQ + h * 16384, h * 64, hkv, k0, b);
           tma_store_4d(&tm_dv, sQ + TB + h * 16384, h * 64, hkv, k0, b);
@@ -556,7 +554,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     if (lane == 0) mbar_wait_drain(mma_final, 0);
     __syncwarp();
     tc_fence_after();

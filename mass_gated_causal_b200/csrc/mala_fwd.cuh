@@ -193,30 +193,29 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      // operand descriptors, built once and stepped with one add per instruction
+      const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dVm = sdesc_sw128(smem_u32(sV), BK * 128, 1024);
       int nv = 0;  // V loads issued (gate on)
       int npv[2] = {0, 0};
       auto issue_qk = [&](int x, int t) {
         const int st = t % NK;
         const uint32_t tS = tmem + Lay::COL_S + x * BK;
+        const uint64_t qa = sdesc_add(dQk, x * Lay::Q_BYTES), kb = sdesc_add(dKk, st * Lay::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a =
-              sdesc_sw128(sQa + x * Lay::Q_BYTES + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd =
-              sdesc_sw128(sKa + st * Lay::KV_BYTES + (kk >> 2) * (BK * 128) + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(tS, a, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16_ss(tS, sdesc_add(qa, (kk >> 2) * (BM * 128) + (kk & 3) * 32),
+                       sdesc_add(kb, (kk >> 2) * (BK * 128) + (kk & 3) * 32), IDESC_QK, kk > 0 ? 1u : 0u);
         umma_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int vslot) {
         const uint32_t tP = tmem + Lay::COL_S + x * BK;  // fp16 P over the first half of S
         const uint32_t tO = tmem + Lay::COL_O + x * D;
+        const uint64_t vb = sdesc_add(dVm, vslot * Lay::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(sVa + vslot * Lay::KV_BYTES + kk * 2048, BK * 128, 1024);
-          umma_f16_ts(tO, tP + kk * 8, bd, IDESC_PV, (npv[x] > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_f16_ts(tO, tP + kk * 8, sdesc_add(vb, kk * 2048), IDESC_PV, (npv[x] > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&pv_done[x]);
         ++npv[x];
       };

@@ -107,6 +107,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Two single-thread waits in one round trip: both phases are tested before
+// either result is needed, so an already complete pair costs one latency.
+__device__ __forceinline__ bool mbar_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1,
+                                           const FailState& fs) {
+  const bool d0 = mbar_try_wait(b0, p0);
+  const bool d1 = mbar_try_wait(b1, p1);
+  if (d0 && d1) return true;
+  return (d0 || mbar_wait(b0, p0, fs)) && (d1 || mbar_wait(b1, p1, fs));
+}
+
 // Warp-uniform bounded wait: every lane returns the same value.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const FailState& fs) {
   bool ok = mbar_try_wait(bar, parity);
@@ -184,6 +194,8 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // the thread's committed bulk copies have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// all but the most recent of the thread's committed bulk groups have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // the thread's committed bulk copies have completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -293,6 +305,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= 1ull << 46;
   d |= 2ull << 61;
   return d;
+}
+
+// A descriptor advanced by a byte offset: the start-address field (bits 0-13)
+// counts 16-byte units and shared addresses stay below 2^18, so the add never
+// carries into the neighbouring fields. Lets the MMA issuer build each
+// operand's descriptor once and step it with one add per instruction.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) {
+  return d + static_cast<uint64_t>(bytes >> 4);
 }
 
 // Instruction descriptor, kind::f16 with fp16 A/B and fp32 D.
