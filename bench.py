@@ -337,8 +337,9 @@ def run_cuda(args):
     t_bwd = fl["bwd"] / (ms_b * 1e-3) / 1e12
     dom = "mala_bwd_kernel" if ms_b >= ms_f else "mala_fwd_kernel"
     ach = t_bwd if dom == "mala_bwd_kernel" else t_fwd
+    traffic = args.traffic if args.traffic is not None else profiled_traffic(dom, w.name)
     roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 2), "peak": peak_t, "unit": "TFLOP/s",
-            "frac": round(ach / peak_t, 4), "traffic": args.traffic,
+            "frac": round(ach / peak_t, 4), "traffic": traffic,
             "peak_kind": f"bf16 dense, {pk['source']} sustained",
             "timed_unit": "mala_bwd call (pre + main + dq convert kernels)" if dom == "mala_bwd_kernel"
             else "mala_fwd call (one kernel)",
@@ -565,6 +566,40 @@ def run_kernel_case(args):
     torch.cuda.synchronize()
     assert mala.mala_check_status() == 0
     print(json.dumps({"kernel_case": args.kernel, "workload": w.name, "ms_mean": e0.elapsed_time(e1) / args.steps}))
+
+
+def kernel_sources_sha256(kernel):
+    """Hash of the sources that define `kernel` (its header and the shared PTX helpers)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "mass_gated_causal_b200", "csrc")
+    name = {"mala_bwd_kernel": "mala_bwd.cuh", "mala_fwd_kernel": "mala_fwd.cuh",
+            "mala_decode_split_kernel": "mala_decode.cuh"}[kernel]
+    h = hashlib.sha256()
+    for f in (name, "mala_ptx.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu summary
+    (profiles/<kernel>_<workload>_dram.md), or None when there is none or when the
+    kernel's sources have changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_dram.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as fh:
+        for line in fh:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("sources-sha256") != kernel_sources_sha256(kernel):
+        return None
+    try:
+        return float(fields["dram-bytes-per-launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def main(argv=None):

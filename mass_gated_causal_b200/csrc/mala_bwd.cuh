@@ -16,22 +16,24 @@
 // mala_bwd_kernel: one CTA owns 128 keys (one key block when Bk = 128, two
 // when Bk = 64) of one (b, KV head) and walks the query tiles of every query
 // head of the GQA group, 128 queries at a time, from the diagonal tile to the
-// end. dK and dV accumulate in TMEM across the whole walk.
-//   warps 0-3  compute: thread t owns query row t of the current tile (TMEM
-//              lane t of S and dP), so its LSE, gate threshold and D are
-//              scalars: gate, P, dS; at the end, key row t of dK and dV
-//   warps 4-7  dQ drain: thread t owns query row t of a kept tile (TMEM lane t
-//              of dQ) and adds it to the fp32 accumulator, while the compute
-//              warps move on to the next tile
-//   warp  8    producer: K, V once; Q tiles and the per-query LSE / threshold
-//              / D vectors through a 2-stage ring
-//   warp  9    MMA issuer: S = Q K^T, then for kept tiles the dO TMA,
-//              dP = dO V^T, dV += P^T dO, the next tile's S, then
-//              dK += dS^T Q and dQ = dS K
-// P and dS share one shared-memory tile (query rows, 128-byte swizzle): dS
-// overwrites P once the dV MMA that reads P^T (MN-major) has finished. dQ
-// reuses the dP TMEM columns and is added to the fp32 accumulator by TMA
-// reduce-add.
+// last, one head after the other. dK and dV accumulate in
+// TMEM across the whole walk. 14 warps:
+//   warps 0-7   compute: thread t owns query row t % 128 of the current tile
+//               and key columns [64h, 64h + 64), h = t / 128 (TMEM lane row of
+//               S and dP), so its LSE, gate threshold and D are scalars: gate,
+//               P (kept in registers), dS; at the end, key row t % 128, half h
+//               of the dK and dV columns
+//   warps 8-11  dQ drain: thread t owns query row t of a kept tile's dQ and
+//               adds it to the fp32 accumulator by TMA reduce-add, while the
+//               compute warps move on
+//   warp  12    producer: K, V once; Q and dO tiles ahead (dO before the gate
+//               has decided: nearly every tile is kept)
+//   warp  13    MMA issuer: S = Q K^T, then for kept tiles dP = dO V^T,
+//               dV += P^T dO, the next tile's S, dK += dS^T Q, dQ = dS K
+// TMEM: two 128-column regions taken by tiles in turn (S, then dP over S,
+// then dQ over dP), then dK and dV. P and dS share one shared-memory tile
+// (query rows, 128-byte swizzle): dS overwrites P once the dV MMA that reads
+// P^T (MN-major) has finished.
 #pragma once
 
 #include "mala_ptx.cuh"
@@ -130,6 +132,12 @@ __global__ void __launch_bounds__(448, 1)
   const int k0 = ks * 128;
   const int nqs = p.n_super - ks;
   const int T = p.G * nqs;
+  // Walk order: the G query heads one after the other, each from the diagonal
+  // query tile to the last. (Walking every CTA of a KV head through the same
+  // tiles in step was measured slower: their dQ additions then hit the same
+  // lines at once.) The backward decisions do not depend on the order.
+  auto walk_hq = [&](int t) { return hkv * p.G + t / nqs; };
+  auto walk_qs = [&](int t) { return ks + t % nqs; };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -178,8 +186,8 @@ __global__ void __launch_bounds__(448, 1)
     for (int t = 0; t < T; ++t) {
       const int st = t & 1;
       if (t >= 2 && !mbar_wait_warp(&q_empty[st], ((t >> 1) - 1) & 1, fs)) break;
-      const int hq = hkv * p.G + t / nqs;
-      const int i0 = (ks + t % nqs) * 128;
+      const int hq = walk_hq(t);
+      const int i0 = walk_qs(t) * 128;
       if (lane == 0) {
         mbar_arrive_expect_tx(&q_full[st], TB);
         for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_q, &q_full[st], sQ + st * TB + h * 16384, h * 64, hq, i0, b);
@@ -240,8 +248,8 @@ __global__ void __launch_bounds__(448, 1)
       if (ok) ok = issue_qk(0);
       for (int t = 0; ok && t < T; ++t) {
         const int st = t & 1;
-        const int hq = hkv * p.G + t / nqs;
-        const int i0 = (ks + t % nqs) * 128;
+        const int hq = walk_hq(t);
+        const int i0 = walk_qs(t) * 128;
         const uint32_t tR = tmem + (t & 1) * 128;
         // the gate's decision (the compute warps have read S(t) out of the
         // region before voting) and dO(t), loaded ahead: one wait for both
@@ -379,18 +387,18 @@ __global__ void __launch_bounds__(448, 1)
     bool local_abort = false, all_abort = false;
     // LSE and D of my row, loaded one tile ahead (rows at or past L: LSE +inf, D 0)
     auto row_lse = [&](int t) {
-      const int i = (ks + t % nqs) * 128 + row;
-      return i < p.L ? __ldg(p.lse + static_cast<size_t>(b * p.Hq + hkv * p.G + t / nqs) * p.L + i) : INFINITY;
+      const int i = walk_qs(t) * 128 + row;
+      return i < p.L ? __ldg(p.lse + static_cast<size_t>(b * p.Hq + walk_hq(t)) * p.L + i) : INFINITY;
     };
     auto row_d = [&](int t) {
-      const int i = (ks + t % nqs) * 128 + row;
-      return i < p.L ? __ldg(p.dvec + static_cast<size_t>(b * p.Hq + hkv * p.G + t / nqs) * p.L + i) : 0.f;
+      const int i = walk_qs(t) * 128 + row;
+      return i < p.L ? __ldg(p.dvec + static_cast<size_t>(b * p.Hq + walk_hq(t)) * p.L + i) : 0.f;
     };
     float lse_next = row_lse(0), d_next = row_d(0);
 
     for (int t = 0; t < T; ++t) {
-      const int hq = hkv * p.G + t / nqs;
-      const int qs = ks + t % nqs;
+      const int hq = walk_hq(t);
+      const int qs = walk_qs(t);
       const bool diag = qs == ks;  // then key column c is live for my row iff c <= row
       const float lse2_row = lse_next * 1.4426950408889634f, d_row = d_next;
       if (t + 1 < T) {

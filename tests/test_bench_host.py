@@ -49,3 +49,19 @@ def test_decode_bytes():
 def test_peaks_present():
     p = bench.peaks()
     assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
+
+
+def test_profiled_traffic_tracks_kernel_sources(tmp_path, monkeypatch):
+    csrc = tmp_path / "mass_gated_causal_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "mala_bwd.cuh").write_text("kernel v1\n")
+    (csrc / "mala_ptx.cuh").write_text("helpers\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("mala_bwd_kernel", "w") is None  # no summary
+    h = bench.kernel_sources_sha256("mala_bwd_kernel")
+    (tmp_path / "profiles" / "mala_bwd_kernel_w_dram.md").write_text(
+        f"# dram\n\n- sources-sha256: `{h}`\n- dram-bytes-per-launch: 1234.5\n")
+    assert bench.profiled_traffic("mala_bwd_kernel", "w") == 1234.5
+    (csrc / "mala_bwd.cuh").write_text("kernel v2\n")  # the kernel changed since the capture
+    assert bench.profiled_traffic("mala_bwd_kernel", "w") is None
