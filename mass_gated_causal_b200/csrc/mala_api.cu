@@ -107,6 +107,22 @@ int set_smem(K kernel, int bytes) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+int sm_count() {
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    sms = 148;
+  return sms;
+}
+
+// Chunk length of the training kernels' CTA schedule: about one wave of CTAs
+// per (b, KV head) unit, but at most a quarter (forward) / half (backward) of
+// a unit's work so that the longest items still start first.
+int fwd_chunk_pairs(int n_pairs, int G) {
+  return std::max(1, std::min(sm_count() / G, (n_pairs + 3) / 4));
+}
+int bwd_chunk_kb(int n_super) { return std::max(1, std::min(sm_count(), (n_super + 1) / 2)); }
+
 // ---------------------------------------------------------------- forward
 template <int D, int BK, bool G>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
@@ -114,7 +130,8 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   using Lay = mala::FwdLayout<D, BK>;
   auto kern = mala::mala_fwd_kernel<D, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(p.n_pairs) * p.B * p.Hq;
+  const unsigned n_chunks = (p.n_pairs + p.chunk_pairs - 1) / p.chunk_pairs;
+  const unsigned grid = n_chunks * p.chunk_pairs * p.B * p.Hq;
   kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
@@ -133,7 +150,8 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   using Lay = mala::BwdLayout<D>;
   auto kern = mala::mala_bwd_kernel<D, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(p.n_super) * p.B * p.Hkv;
+  const unsigned n_chunks = (p.n_super + p.chunk_kb - 1) / p.chunk_kb;
+  const unsigned grid = n_chunks * p.chunk_kb * p.B * p.Hkv;
   kern<<<grid, 448, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
@@ -219,6 +237,7 @@ int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.nq = (L + Bq - 1) / Bq;
   p.nk = (L + Bk - 1) / Bk;
   p.n_pairs = (L + 255) / 256;
+  p.chunk_pairs = fwd_chunk_pairs(p.n_pairs, p.G);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;
   p.lse = lse;
@@ -273,6 +292,7 @@ int mala_bwd(const void* q, const void* k, const void* v, const void* o, const v
   p.nq = (L + Bq - 1) / Bq;
   p.nk = (L + Bk - 1) / Bk;
   p.n_super = (L + 127) / 128;
+  p.chunk_kb = bwd_chunk_kb(p.n_super);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;

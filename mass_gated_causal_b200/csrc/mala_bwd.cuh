@@ -43,6 +43,7 @@ namespace mala {
 struct BwdParams {
   int B, Hq, Hkv, L, G;
   int nq, nk, n_super;
+  int chunk_kb;  // CTA schedule: key blocks per chunk (see mala_bwd_kernel)
   float scale, scale_log2, log2_tau;
   const float* lse;   // [B, Hq, L]
   const float* dvec;  // [B, Hq, L]: D_i
@@ -125,9 +126,17 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nbk = p.B * p.Hkv;
-  const int bk = blockIdx.x % nbk;
-  const int ks = static_cast<int>(blockIdx.x / nbk);  // ascending: longest walks first
+  // CTA schedule: the grid is cut into chunks of chunk_kb key blocks, longest
+  // walks (lowest key blocks) first; inside a chunk the (b, KV head) units
+  // follow one another. The CTAs resident at one time then read the Q / dO
+  // tiles and add into the dQ rows of one or two KV heads' query heads, which
+  // stay in L2. The last chunk may be padded with empty CTAs.
+  const int per_chunk = p.B * p.Hkv * p.chunk_kb;
+  const int chunk = static_cast<int>(blockIdx.x) / per_chunk;
+  const int in_chunk = static_cast<int>(blockIdx.x) % per_chunk;
+  const int bk = in_chunk / p.chunk_kb;
+  const int ks = chunk * p.chunk_kb + in_chunk % p.chunk_kb;
+  if (ks >= p.n_super) return;  // padding (uniform across the CTA, before any shared state)
   const int b = bk / p.Hkv, hkv = bk % p.Hkv;
   const int k0 = ks * 128;
   const int nqs = p.n_super - ks;

@@ -37,6 +37,7 @@ namespace mala {
 struct FwdParams {
   int B, Hq, Hkv, L, G;
   int nq, nk, n_pairs;  // n_pairs = ceil(L / 256) pairs of 128-row tiles
+  int chunk_pairs;      // CTA schedule: pairs per chunk (see mala_fwd_kernel)
   float scale_log2;     // scale * log2(e): scores are kept in log2 units
   float log2_tau;       // log2(tau), used only when the gate is on
   float* lse;           // [B, Hq, L]
@@ -121,10 +122,20 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nbh = p.B * p.Hq;
-  const int bh = blockIdx.x % nbh;
-  const int pr = p.n_pairs - 1 - static_cast<int>(blockIdx.x / nbh);  // longest rows first
-  const int b = bh / p.Hq, hq = bh % p.Hq, hkv = hq / p.G;
+  // CTA schedule: the grid is cut into chunks of chunk_pairs row pairs, longest
+  // rows first; inside a chunk the (b, KV head) units follow one another and the
+  // G query heads of a pair are adjacent. The CTAs resident at one time then
+  // share one or two KV heads, whose K and V stay in L2, while the longest
+  // rows still start first. The last chunk may be padded with empty CTAs.
+  const int per_unit = p.chunk_pairs * p.G;
+  const int per_chunk = p.B * p.Hkv * per_unit;
+  const int chunk = static_cast<int>(blockIdx.x) / per_chunk;
+  const int in_chunk = static_cast<int>(blockIdx.x) % per_chunk;
+  const int unit = in_chunk / per_unit;
+  const int pr = p.n_pairs - 1 - (chunk * p.chunk_pairs + (in_chunk % per_unit) / p.G);
+  if (pr < 0) return;  // padding (uniform across the CTA, before any shared state)
+  const int b = unit / p.Hkv, hkv = unit % p.Hkv, hq = hkv * p.G + in_chunk % p.G;
+  const int bh = b * p.Hq + hq;
   const int r0 = pr * 2 * BM;  // first row of tile A
   const int last_row = min(r0 + 2 * BM, p.L) - 1;
   const int kb_hi = last_row / BK;
