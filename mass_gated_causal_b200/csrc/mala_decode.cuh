@@ -278,16 +278,17 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int LPH = LPK / GP;  // lanes of a key row that end up holding the same head
   const int hh = c / LPH;        // the head whose scores this lane holds after the reduction
   const bool owner = kg == 0 && (c % LPH) == 0;  // writes head hh's per-warp statistics
-  float qr[GP][8];
+  // q slice and output accumulators as packed fp32 pairs (elements e, e+1)
+  uint64_t qr[GP][4];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) qr[g][e] = sq[g * D + c * 8 + e];
-  float acc[GP][8];
+    for (int e2 = 0; e2 < 4; ++e2) qr[g][e2] = f2_pack(sq[g * D + c * 8 + 2 * e2], sq[g * D + c * 8 + 2 * e2 + 1]);
+  uint64_t acc[GP][4];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+    for (int e2 = 0; e2 < 4; ++e2) acc[g][e2] = 0ull;  // (+0, +0)
   float ring[NP][STEPS];  // probabilities of pending kept tiles (head hh of each step's key)
 #pragma unroll
   for (int i = 0; i < NP; ++i)
@@ -313,14 +314,20 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int g = 0; g < GP; ++g) part[g] = 0.f;
       if (okk) {
-        uint32_t a0, a1, a2, a3;
-        ld_shared_v4(row_addr(sKa + st * TB, j), a0, a1, a2, a3);
-        const float kf[8] = {bf16lo_to_f32(a0), bf16hi_to_f32(a0), bf16lo_to_f32(a1), bf16hi_to_f32(a1),
-                             bf16lo_to_f32(a2), bf16hi_to_f32(a2), bf16lo_to_f32(a3), bf16hi_to_f32(a3)};
+        uint32_t a[4];
+        ld_shared_v4(row_addr(sKa + st * TB, j), a[0], a[1], a[2], a[3]);
+        uint64_t kf[4];
 #pragma unroll
-        for (int g = 0; g < GP; ++g)
+        for (int e2 = 0; e2 < 4; ++e2) kf[e2] = bf16x2_to_f2(a[e2]);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) part[g] = fmaf(kf[e], qr[g][e], part[g]);
+        for (int g = 0; g < GP; ++g) {
+          uint64_t s2 = f2_fma(kf[0], qr[g][0], 0ull);  // even / odd elements summed separately
+#pragma unroll
+          for (int e2 = 1; e2 < 4; ++e2) s2 = f2_fma(kf[e2], qr[g][e2], s2);
+          float lo, hi;
+          f2_unpack(s2, lo, hi);
+          part[g] = lo + hi;
+        }
       }
       const float mine = group_reduce_scatter<GP, LPK>(part, c);  // score of key j for my head hh
       const bool live = kb * BK + j < p.Lk;
@@ -342,21 +349,24 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       const float al = sAlpha[ps * GP + g];
+      const uint64_t al2 = f2_pack(al, al);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] *= al;
+      for (int e2 = 0; e2 < 4; ++e2) acc[g][e2] = f2_mul(acc[g][e2], al2);
     }
 #pragma unroll
     for (int s2 = 0; s2 < STEPS; ++s2) {
       const int j = warp * KPWT + s2 * KPW + kg;
-      uint32_t a0, a1, a2, a3;
-      ld_shared_v4(row_addr(sVa + vs * TB, j), a0, a1, a2, a3);
-      const float vf[8] = {bf16lo_to_f32(a0), bf16hi_to_f32(a0), bf16lo_to_f32(a1), bf16hi_to_f32(a1),
-                           bf16lo_to_f32(a2), bf16hi_to_f32(a2), bf16lo_to_f32(a3), bf16hi_to_f32(a3)};
+      uint32_t a[4];
+      ld_shared_v4(row_addr(sVa + vs * TB, j), a[0], a[1], a[2], a[3]);
+      uint64_t vf[4];
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) vf[e2] = bf16x2_to_f2(a[e2]);
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         const float pg = __shfl_sync(0xffffffffu, pr[s2], kg * LPK + g * LPH);
+        const uint64_t pg2 = f2_pack(pg, pg);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
+        for (int e2 = 0; e2 < 4; ++e2) acc[g][e2] = f2_fma(pg2, vf[e2], acc[g][e2]);
       }
     }
   };
@@ -407,17 +417,22 @@ __global__ void __launch_bounds__(320, 1)
   }
   named_bar_sync(2, NT);  // compute warps only (barrier 2): every read of the rings is done
   float* ored = reinterpret_cast<float*>(sK);  // [NW][GP][D], reuses the K ring
+  float accf[GP][8];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) f2_unpack(acc[g][e2], accf[g][2 * e2], accf[g][2 * e2 + 1]);
 #pragma unroll
   for (int off = LPK; off < 32; off <<= 1)  // sum the key groups of the warp
 #pragma unroll
     for (int g = 0; g < GP; ++g)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], off);
+      for (int e = 0; e < 8; ++e) accf[g][e] += __shfl_xor_sync(0xffffffffu, accf[g][e], off);
   if (kg == 0) {
 #pragma unroll
     for (int g = 0; g < GP; ++g)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ored[(warp * GP + g) * D + c * 8 + e] = acc[g][e];
+      for (int e = 0; e < 8; ++e) ored[(warp * GP + g) * D + c * 8 + e] = accf[g][e];
   }
   named_bar_sync(1, NB);  // D (with the gate warp, which has folded the last sums into sL)
   if (!aborted && !abort_raised(fs)) {
