@@ -54,6 +54,9 @@ def _load():
         lib.oracle_fwd.argtypes = [_dp, _dp, _dp, i, i, i, i, i, d_, d_, i, i, _i32p, i,
                                    _dp, _dp, _u8p, _dp, _i64p]
         lib.oracle_fwd.restype = None
+        lib.oracle_prefill.argtypes = [_dp, _dp, _dp, i, i, i, i, i, i, d_, d_, i, i, _i32p, i,
+                                       _dp, _dp, _u8p, _dp, _i64p]
+        lib.oracle_prefill.restype = None
         lib.oracle_dense_lse.argtypes = [_dp, _dp, i, i, i, i, i, d_, _dp]
         lib.oracle_dense_lse.restype = None
         lib.oracle_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, i, i, i, i, i, d_, d_, i, i,
@@ -119,6 +122,35 @@ def fwd(q, k, v, scale: float, tau: float, Bq: int, Bk: int,
     _load().oracle_fwd(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), B, Hq, Hkv, L, d, float(scale),
                        float(tau), Bq, Bk, _ptr(s, _i32p), ns, _ptr(o, _dp), _ptr(lse, _dp),
                        _ptr(keep, _u8p), _ptr(margin, _dp), _ptr(kept, _i64p))
+    return {"o": o, "lse": lse, "keep": keep, "margin": margin, "kept": kept}
+
+
+def prefill(q, k, v, scale: float, tau: float, Bq: int, Bk: int,
+            sel: Optional[Sequence] = None, with_margin: bool = True):
+    """MALA forward of Lq new queries against Lk >= Lq keys (prefill against an
+    existing cache). q [B,Lq,Hq,d] holds the queries at positions Lk-Lq ..
+    Lk-1; k/v [B,Lk,Hkv,d] (fp64). Query blocks start at the first new query.
+
+    Returns dict with o [B,Lq,Hq,d], lse [B,Hq,Lq], keep [B,Hq,nq,nk]
+    (nq = ceil(Lq/Bq), nk = ceil(Lk/Bk)), margin, kept [B*Hq]; ``sel`` as in fwd.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    assert Lk >= Lq
+    nq, nk = -(-Lq // Bq), -(-Lk // Bk)
+    o = np.full_like(q, np.nan)
+    lse = np.full((B, Hq, Lq), np.nan)
+    keep = np.full((B, Hq, nq, nk), 255 if sel is not None else 0, dtype=np.uint8)
+    margin = np.full((B, Hq, nq, nk), np.nan) if with_margin else None
+    kept = np.zeros(B * Hq, dtype=np.int64)
+    s, ns = _sel(sel, 3)
+    if sel is not None:
+        for (b, hq, qb) in s:
+            keep[b, hq, qb] = 0
+    _load().oracle_prefill(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), B, Hq, Hkv, Lq, Lk, d, float(scale),
+                           float(tau), Bq, Bk, _ptr(s, _i32p), ns, _ptr(o, _dp), _ptr(lse, _dp),
+                           _ptr(keep, _u8p), _ptr(margin, _dp), _ptr(kept, _i64p))
     return {"o": o, "lse": lse, "keep": keep, "margin": margin, "kept": kept}
 
 

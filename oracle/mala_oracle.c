@@ -36,6 +36,13 @@
  *      partial results are merged by their LSEs;
  *   R8 GQA: decisions are per query head.
  *
+ * Prefill against an existing cache (oracle_prefill): Lq new queries at the
+ * positions Lk - Lq, ..., Lk - 1 of a sequence of Lk keys; row i (0-based
+ * among the new queries) sees keys 0 .. P0 + i, P0 = Lk - Lq, and its
+ * threshold uses Lq_i = P0 + i + 1 (the count of causally visible keys); the
+ * query blocks are cut from the first new query. With Lq == Lk it is the
+ * forward above.
+ *
  * Layouts: q, o, dO, dq [B, L, Hq, d]; k, v, dk, dv [B, L, Hkv, d];
  * lse [B, Hq, L] (natural log); keep maps [B, Hq, nq, nk] (1 kept, 0 skipped
  * or illegal); margins [B, Hq, nq, nk] (g = max over rows of ratio/(tau/Lq),
@@ -82,21 +89,35 @@ static double score(const double* q, const double* k, int b, int i, int j, int h
     return scale * acc;
 }
 
+/* s = scale * <q[b, i, hq, :], k[b, j, hkv, :]> with q holding Lq rows and k
+ * holding Lk rows (prefill) */
+static double score2(const double* q, const double* k, int b, int i, int j, int hq, int hkv,
+                     int Lq, int Lk, int Hq, int Hkv, int d, double scale) {
+    const double* qi = q + IDX4(b, i, hq, 0, Lq, Hq, d);
+    const double* kj = k + IDX4(b, j, hkv, 0, Lk, Hkv, d);
+    double acc = 0.0;
+    for (int c = 0; c < d; ++c) acc += qi[c] * kj[c];
+    return scale * acc;
+}
+
 /* ------------------------------------------------------------------------
- * Forward: one query block (b, hq, qb).
+ * Forward: one query block (b, hq, qb) of Lq queries at positions P0 + i
+ * (P0 = Lk - Lq) against Lk keys; P0 = 0 is the training forward.
  * ---------------------------------------------------------------------- */
 static void fwd_block(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
-                      int L, int d, double scale, double tau, int Bq, int Bk, int b, int hq, int qb,
-                      double* o, double* lse, uint8_t* keep_map, double* margin, int64_t* n_kept) {
+                      int Lq, int Lk, int d, double scale, double tau, int Bq, int Bk, int b, int hq,
+                      int qb, double* o, double* lse, uint8_t* keep_map, double* margin,
+                      int64_t* n_kept) {
     (void)B;
     const int G = Hq / Hkv;
     const int hkv = hq / G;
-    const int nq = (L + Bq - 1) / Bq;
-    const int nk = (L + Bk - 1) / Bk;
+    const int P0 = Lk - Lq;
+    const int nq = (Lq + Bq - 1) / Bq;
+    const int nk = (Lk + Bk - 1) / Bk;
     const int i0 = qb * Bq;
-    const int i1 = imin((qb + 1) * Bq, L); /* rows [i0, i1) */
+    const int i1 = imin((qb + 1) * Bq, Lq); /* rows [i0, i1) among the new queries */
     const int R = i1 - i0;
-    const int kb_first = (i1 - 1) / Bk;    /* largest legal key block */
+    const int kb_first = (P0 + i1 - 1) / Bk; /* largest legal key block */
 
     double* m = (double*)malloc(sizeof(double) * R);
     double* l = (double*)malloc(sizeof(double) * R);
@@ -107,21 +128,21 @@ static void fwd_block(const double* q, const double* k, const double* v, int B, 
     for (int r = 0; r < R; ++r) {
         m[r] = -INFINITY;
         l[r] = 0.0;
-        thr[r] = tau > 0.0 ? log(tau) - log((double)(i0 + r + 1)) : -INFINITY; /* ln(tau/Lq) */
+        thr[r] = tau > 0.0 ? log(tau) - log((double)(P0 + i0 + r + 1)) : -INFINITY; /* ln(tau/Lq) */
     }
     int64_t kept = 0;
     size_t map_row = ((size_t)(b * Hq + hq) * nq + qb) * nk;
 
     for (int kb = kb_first; kb >= 0; --kb) { /* diagonal toward earlier keys */
         const int j0 = kb * Bk;
-        const int j1 = imin((kb + 1) * Bk, L);
+        const int j1 = imin((kb + 1) * Bk, Lk);
         /* 1. scores of every live entry of the tile (never skipped) */
         for (int r = 0; r < R; ++r) {
             const int i = i0 + r;
             M[r] = -INFINITY;
             for (int j = j0; j < j1; ++j) {
                 double sv = -INFINITY;
-                if (j <= i) sv = score(q, k, b, i, j, hq, hkv, L, Hq, Hkv, d, scale);
+                if (j <= P0 + i) sv = score2(q, k, b, i, j, hq, hkv, Lq, Lk, Hq, Hkv, d, scale);
                 s[(size_t)r * Bk + (j - j0)] = sv;
                 if (sv > M[r]) M[r] = sv;
             }
@@ -162,7 +183,7 @@ static void fwd_block(const double* q, const double* k, const double* v, int B, 
                 if (sv == -INFINITY) continue;
                 const double p = exp(sv - mn);
                 l[r] += p;
-                const double* vj = v + IDX4(b, j, hkv, 0, L, Hkv, d);
+                const double* vj = v + IDX4(b, j, hkv, 0, Lk, Hkv, d);
                 for (int c = 0; c < d; ++c) ar[c] += p * vj[c];
             }
             m[r] = mn;
@@ -171,25 +192,27 @@ static void fwd_block(const double* q, const double* k, const double* v, int B, 
     /* 4. O = acc / l, LSE = m + ln l */
     for (int r = 0; r < R; ++r) {
         const int i = i0 + r;
-        double* oi = o + IDX4(b, i, hq, 0, L, Hq, d);
+        double* oi = o + IDX4(b, i, hq, 0, Lq, Hq, d);
         for (int c = 0; c < d; ++c) oi[c] = acc[(size_t)r * d + c] / l[r];
-        lse[((size_t)b * Hq + hq) * L + i] = m[r] + log(l[r]);
+        lse[((size_t)b * Hq + hq) * Lq + i] = m[r] + log(l[r]);
     }
     *n_kept = kept;
     free(m); free(l); free(thr); free(acc); free(s); free(M);
 }
 
 /*
- * oracle_fwd: MALA forward over all query blocks (sel == NULL) or over the
+ * oracle_prefill: MALA forward of Lq queries against Lk >= Lq keys (see the
+ * header), over all query blocks (sel == NULL) or over the
  * nsel blocks listed in sel as (b, hq, qb) triples. Only the selected rows of
  * o / lse and the selected rows of keep_map / margin are written; kept_tiles
  * receives the number of kept tiles per (b, hq) over the selected blocks.
  * keep_map, margin and kept_tiles may be NULL.
  */
-void oracle_fwd(const double* q, const double* k, const double* v, int B, int Hq, int Hkv, int L,
-                int d, double scale, double tau, int Bq, int Bk, const int32_t* sel, int nsel,
-                double* o, double* lse, uint8_t* keep_map, double* margin, int64_t* kept_tiles) {
-    const int nq = (L + Bq - 1) / Bq;
+void oracle_prefill(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
+                    int Lq, int Lk, int d, double scale, double tau, int Bq, int Bk,
+                    const int32_t* sel, int nsel, double* o, double* lse, uint8_t* keep_map,
+                    double* margin, int64_t* kept_tiles) {
+    const int nq = (Lq + Bq - 1) / Bq;
     const long total = sel ? (long)nsel : (long)B * Hq * nq;
     int64_t* per = (int64_t*)calloc((size_t)(total > 0 ? total : 1), sizeof(int64_t));
 #pragma omp parallel for schedule(dynamic, 1)
@@ -204,7 +227,7 @@ void oracle_fwd(const double* q, const double* k, const double* v, int B, int Hq
             u %= (long)B * Hq;
             b = (int)(u / Hq); hq = (int)(u % Hq);
         }
-        fwd_block(q, k, v, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, b, hq, qb, o, lse, keep_map,
+        fwd_block(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, tau, Bq, Bk, b, hq, qb, o, lse, keep_map,
                   margin, &per[t]);
     }
     if (kept_tiles) {
@@ -217,6 +240,14 @@ void oracle_fwd(const double* q, const double* k, const double* v, int B, int Hq
         }
     }
     free(per);
+}
+
+/* oracle_fwd: the training forward (queries and keys of one sequence). */
+void oracle_fwd(const double* q, const double* k, const double* v, int B, int Hq, int Hkv, int L,
+                int d, double scale, double tau, int Bq, int Bk, const int32_t* sel, int nsel,
+                double* o, double* lse, uint8_t* keep_map, double* margin, int64_t* kept_tiles) {
+    oracle_prefill(q, k, v, B, Hq, Hkv, L, L, d, scale, tau, Bq, Bk, sel, nsel, o, lse, keep_map,
+                   margin, kept_tiles);
 }
 
 /*

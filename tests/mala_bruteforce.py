@@ -168,3 +168,58 @@ def bf_decode(q, kc, vc, scale, tau, Bk, n_splits):
             for c in range(d):
                 o[b, hq, c] = float(mp.fsum(E[j] * mp.mpf(float(vc[b, j, hkv, c])) for j in allkept) / Z)
     return {"o": o, "lse": lse, "keep": keep}
+
+
+def bf_prefill(q, k, v, scale, tau, Bq, Bk):
+    """Forward of Lq new queries at positions P0 + i (P0 = Lk - Lq) against Lk
+    keys, with query blocks cut from the first new query and thresholds
+    tau / (P0 + i + 1). Explicit kept-key sets, unstabilised ratios."""
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    P0 = Lk - Lq
+    G = Hq // Hkv
+    nq, nk = -(-Lq // Bq), -(-Lk // Bk)
+    tau_m = mp.mpf(tau)
+    sc = mp.mpf(scale)
+    keep = np.zeros((B, Hq, nq, nk), dtype=np.uint8)
+    o = np.zeros(q.shape)
+    lse = np.zeros((B, Hq, Lq))
+    for b in range(B):
+        for hq in range(Hq):
+            hkv = hq // G
+            E = {}
+            for i in range(Lq):
+                qi = [mp.mpf(float(x)) for x in q[b, i, hq]]
+                for j in range(P0 + i + 1):
+                    E[(i, j)] = mp.exp(sc * mp.fsum(qi[c] * mp.mpf(float(k[b, j, hkv, c])) for c in range(d)))
+            for qb in range(nq):
+                rows = range(qb * Bq, min((qb + 1) * Bq, Lq))
+                sets = {i: set() for i in rows}
+                kb_first = (P0 + max(rows)) // Bk
+                for kb in range(kb_first, -1, -1):
+                    keys = range(kb * Bk, min((kb + 1) * Bk, Lk))
+                    if kb == kb_first or tau == 0:
+                        kp = True
+                    else:
+                        kp = False
+                        for i in rows:
+                            live = [j for j in keys if j <= P0 + i]
+                            if not live:
+                                continue
+                            if not sets[i]:
+                                kp = True
+                                continue
+                            Z = mp.fsum(E[(i, j)] for j in sets[i])
+                            if any(E[(i, j)] / Z >= tau_m / (P0 + i + 1) for j in live):
+                                kp = True
+                    keep[b, hq, qb, kb] = 1 if kp else 0
+                    if kp:
+                        for i in rows:
+                            sets[i].update(j for j in keys if j <= P0 + i)
+                for i in rows:
+                    Z = mp.fsum(E[(i, j)] for j in sets[i])
+                    lse[b, hq, i] = float(mp.log(Z))
+                    for c in range(d):
+                        o[b, i, hq, c] = float(mp.fsum(E[(i, j)] * mp.mpf(float(v[b, j, hkv, c]))
+                                                       for j in sets[i]) / Z)
+    return {"o": o, "lse": lse, "keep": keep}

@@ -20,14 +20,18 @@ from workloads import TrainWorkload, bf16_bits_to_f64, make_train_inputs
 
 MUTANTS = {
     "drop_rescale_of_acc": ("for (int c = 0; c < d; ++c) ar[c] *= alpha;", ""),
-    "lq_off_by_one": ("log((double)(i0 + r + 1))", "log((double)(i0 + r))"),
+    "lq_off_by_one": ("log((double)(P0 + i0 + r + 1))", "log((double)(P0 + i0 + r))"),
+    "prefill_lq_ignores_offset": ("log((double)(P0 + i0 + r + 1))", "log((double)(i0 + r + 1))"),
+    "prefill_first_tile_ignores_offset": ("const int kb_first = (P0 + i1 - 1) / Bk;",
+                                          "const int kb_first = (i1 - 1) / Bk;"),
+    "prefill_live_ignores_offset": ("if (j <= P0 + i) sv", "if (j <= i) sv"),
     "visit_order_reversed": ("for (int kb = kb_first; kb >= 0; --kb)", "for (int kb = 0; kb <= kb_first; ++kb)"),
     "gate_uses_max_not_ratio": ("(M[r] - m[r] - log(l[r])) - thr[r]", "(M[r] - m[r]) - thr[r]"),
     "ds_sign": ("const double dS = P * (dP - Di);\n                    for (int c = 0; c < d; ++c) dqi",
                 "const double dS = P * (dP + Di);\n                    for (int c = 0; c < d; ++c) dqi"),
     "dq_drops_scale": ("dqi[c] += scale * dS * kj[c];", "dqi[c] += dS * kj[c];"),
     "bwd_gate_sign": ("- LSEi - thr;", "- LSEi + thr;"),
-    "gqa_head_map": ("const int hkv = hq / G;\n    const int nq", "const int hkv = hq % Hkv;\n    const int nq"),
+    "gqa_head_map": ("const int hkv = hq / G;\n    const int P0", "const int hkv = hq % Hkv;\n    const int P0"),
     "dk_uses_k_not_q": ("dkj[c] += scale * dS * qi[c];", "dkj[c] += scale * dS * gi[c];"),
     "decode_forces_oldest": ("if (kb == t1 - 1) keep = 1;", "if (kb == t0) keep = 1;"),
     "decode_lq_is_split_length": ("log((double)Lk)", "log((double)(Lk / n_splits + 1))"),
@@ -72,6 +76,15 @@ def _pins_pass() -> bool:
             return False
         for name in ("dq", "dk", "dv"):
             if np.abs(g[name] - rb[name]).max() > 1e-8:
+                return False
+        # prefill against a cache (offset not a multiple of Bq, Bq != Bk) vs the brute force
+        q, k, v, _ = _case(44, 8, 2, 1, 41, 1.5)
+        for (tau, Bq, Bk) in ((1.0, 8, 4), (4.0, 4, 8)):
+            r = oracle.prefill(q[:, 23:], k, v, sc, tau, Bq, Bk)
+            rp = bf.bf_prefill(q[:, 23:], k, v, sc, tau, Bq, Bk)
+            if not (r["keep"] == rp["keep"]).all() or np.abs(r["o"] - rp["o"]).max() > 1e-9:
+                return False
+            if np.abs(r["lse"] - rp["lse"]).max() > 1e-9:
                 return False
         # decode vs the brute force
         q, k, v, _ = _case(50, 8, 2, 1, 31, 2.0)
