@@ -22,8 +22,9 @@
  *     the host before anything is enqueued: on any error return nothing is
  *     written and nothing is launched.
  *   - GQA: query head hq reads KV head hq / (Hq / Hkv).
- *   - Supported: d in {64, 128}; Bq == Bk in {64, 128}; any L >= 1 (a ragged
- *     last tile is fine); B, Hq, Hkv >= 1 with Hq % Hkv == 0.
+ *   - Supported: d in {64, 128}; Bq and Bk each in {64, 128} (independently);
+ *     any L >= 1 (a ragged last tile is fine); B, Hq, Hkv >= 1 with
+ *     Hq % Hkv == 0.
  *   - Device-side waits are bounded. If one expires the kernel records
  *     MALA_ERR_DEVICE_TIMEOUT in a device status word and returns;
  *     mala_check_status() reports it.
@@ -101,9 +102,40 @@ MALA_API int mala_fwd(const void* q, const void* k, const void* v, void* o, floa
 
 /*
  * Workspace bytes mala_fwd needs: the fp16 copy of V [B, L, Hkv, d] the PV
- * product reads (256-byte aligned). Returns 0 for invalid sizes.
+ * product reads (256-byte aligned). Returns 0 for invalid sizes. mala_prefill
+ * needs mala_fwd_workspace_size(B, Hkv, Lk, d).
  */
 MALA_API size_t mala_fwd_workspace_size(int B, int Hkv, int L, int d);
+
+/*
+ * mala_prefill -- MALA forward of Lq new queries against Lk >= Lq keys (a
+ * prompt chunk appended to an existing KV cache).
+ *
+ * Source: agihunt.info MALA digest, method paragraphs (the forward gate, with
+ * Lq the number of keys the query sees) and limitations paragraph (the KV
+ * cache is kept whole; one tau for training and serving).
+ *
+ * The new queries sit at the end of the sequence: query row i (0 <= i < Lq)
+ * is at position P0 + i with P0 = Lk - Lq, sees keys 0 .. P0 + i and uses the
+ * threshold tau / (P0 + i + 1). Query blocks are cut from the first new
+ * query (block qb = rows [qb*Bq, min((qb+1)*Bq, Lq))); key blocks from key 0.
+ * Tile (qb, kb) is legal iff kb*Bk <= P0 + min((qb+1)*Bq, Lq) - 1, and the
+ * block's first legal tile is the one holding that key. Everything else
+ * (visit order, forced first tile, the gate, LSE) is as in mala_fwd; with
+ * Lq == Lk the call computes exactly what mala_fwd does.
+ *
+ *   q          [B, Lq, Hq, d]  bf16, in
+ *   k, v       [B, Lk, Hkv, d] bf16, in (the cache with the new keys at the end)
+ *   o          [B, Lq, Hq, d]  bf16, out
+ *   lse        [B, Hq, Lq]     fp32, out (natural log)
+ *   Lq >= 1, Lk >= Lq; other arguments as for mala_fwd, with nq = ceil(Lq/Bq),
+ *   nk = ceil(Lk/Bk) for keep_map [B, Hq, nq, nk]
+ *   workspace  >= mala_fwd_workspace_size(B, Hkv, Lk, d) bytes
+ * Errors: MALA_ERR_INVALID_ARG also for Lq < 1 or Lk < Lq.
+ */
+MALA_API int mala_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Lq, int Lk, int d, float scale, float tau, int Bq, int Bk, void* workspace,
+             size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
 
 /*
  * Workspace bytes mala_bwd needs: an fp32 dQ accumulator [B, L, Hq, d] and

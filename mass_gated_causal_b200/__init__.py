@@ -5,9 +5,9 @@ this module only turns torch tensors into device pointers, allocates outputs
 with torch and passes the current CUDA stream. There is no CPU fallback: if the
 library is missing, importing this package raises.
 
-Raw entry points keep the C names (``mala_fwd``, ``mala_bwd``, ``mala_decode``,
-...). ``forward``, ``backward`` and ``decode`` are conveniences that allocate
-the outputs and workspaces.
+Raw entry points keep the C names (``mala_fwd``, ``mala_prefill``, ``mala_bwd``,
+``mala_decode``, ...). ``forward``, ``prefill``, ``backward`` and ``decode`` are
+conveniences that allocate the outputs and workspaces.
 """
 from __future__ import annotations
 
@@ -33,7 +33,8 @@ MALA_ERR_CUDA = 4
 MALA_ERR_DEVICE_TIMEOUT = 5
 MALA_ERR_RANGE = 6
 
-EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_fwd_workspace_size", "mala_bwd_workspace_size",
+EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_prefill", "mala_fwd_workspace_size",
+            "mala_bwd_workspace_size",
             "mala_bwd",
             "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_noalloc_max_bytes",
             "mala_decode_noalloc", "mala_check_status")
@@ -44,6 +45,9 @@ _lib.mala_status_string.restype = ctypes.c_char_p
 _lib.mala_abi_version.restype = _i
 _lib.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp, _vp]
 _lib.mala_fwd.restype = _i
+_lib.mala_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp,
+                              _vp]
+_lib.mala_prefill.restype = _i
 _lib.mala_fwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.mala_fwd_workspace_size.restype = _sz
 _lib.mala_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
@@ -110,6 +114,13 @@ def mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace, w
                              _stream(stream)))
 
 
+def mala_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, tau, Bq, Bk, workspace, workspace_bytes,
+                 kept_tiles, keep_map=None, stream=None) -> int:
+    return int(_lib.mala_prefill(_p(q), _p(k), _p(v), _p(o), _p(lse), B, Hq, Hkv, Lq, Lk, d, float(scale),
+                                 float(tau), Bq, Bk, _p(workspace), int(workspace_bytes), _p(kept_tiles),
+                                 _p(keep_map), _stream(stream)))
+
+
 def mala_fwd_workspace_size(B, Hkv, L, d) -> int:
     return int(_lib.mala_fwd_workspace_size(B, Hkv, L, d))
 
@@ -172,6 +183,27 @@ def forward(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, kee
         km = torch.full((B, Hq, -(-L // Bq), -(-L // Bk)), 255, dtype=torch.uint8, device=q.device)
     _check(mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace,
                     workspace.numel() * workspace.element_size(), kept, km, stream), "mala_fwd")
+    return o, lse, kept, km
+
+
+def prefill(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, keep_map: bool = False,
+            workspace=None, stream=None):
+    """q [B,Lq,Hq,d] (new queries), k/v [B,Lk,Hkv,d] (cache incl. the new keys)
+    -> (o [B,Lq,Hq,d], lse [B,Hq,Lq], kept_tiles, keep_map|None)."""
+    import torch
+    B, Lq, Hq, d = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    if workspace is None:
+        workspace = torch.empty((max(1, mala_fwd_workspace_size(B, Hkv, Lk, d)),), dtype=torch.uint8,
+                                device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    kept = torch.empty((B * Hq,), dtype=torch.int32, device=q.device)
+    km = None
+    if keep_map:
+        km = torch.full((B, Hq, -(-Lq // Bq), -(-Lk // Bk)), 255, dtype=torch.uint8, device=q.device)
+    _check(mala_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, tau, Bq, Bk, workspace,
+                        workspace.numel() * workspace.element_size(), kept, km, stream), "mala_prefill")
     return o, lse, kept, km
 
 

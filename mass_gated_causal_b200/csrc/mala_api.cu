@@ -91,7 +91,7 @@ int check_train_shape(int B, int Hq, int Hkv, int L, int d, float scale, float t
   if (!(scale > 0.f) || !std::isfinite(scale)) return MALA_ERR_INVALID_ARG;
   if (!(tau >= 0.f) || !std::isfinite(tau)) return MALA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
-  if (Bq != Bk || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
+  if ((Bq != 64 && Bq != 128) || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
   // element counts must fit the int arithmetic of the kernels
   if (static_cast<long long>(B) * L * Hq * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Hq >= (1ll << 24)) return MALA_ERR_UNSUPPORTED;
@@ -124,11 +124,11 @@ int fwd_chunk_pairs(int n_pairs, int G) {
 int bwd_chunk_kb(int n_super) { return std::max(1, std::min(sm_count(), (n_super + 1) / 2)); }
 
 // ---------------------------------------------------------------- forward
-template <int D, int BK, bool G>
+template <int D, int BQ, int BK, bool G>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                const mala::FwdParams& p, cudaStream_t st) {
   using Lay = mala::FwdLayout<D, BK>;
-  auto kern = mala::mala_fwd_kernel<D, BK, G>;
+  auto kern = mala::mala_fwd_kernel<D, BQ, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned n_chunks = (p.n_pairs + p.chunk_pairs - 1) / p.chunk_pairs;
   const unsigned grid = n_chunks * p.chunk_pairs * p.B * p.Hq;
@@ -136,19 +136,29 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
-template <int D, int BK>
+template <int D, int BQ, int BK>
 int launch_fwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mo, const mala::FwdParams& p, cudaStream_t st) {
-  return gate ? launch_fwd<D, BK, true>(mq, mk, mv, mo, p, st) : launch_fwd<D, BK, false>(mq, mk, mv, mo, p, st);
+  return gate ? launch_fwd<D, BQ, BK, true>(mq, mk, mv, mo, p, st)
+              : launch_fwd<D, BQ, BK, false>(mq, mk, mv, mo, p, st);
+}
+
+template <int D>
+int launch_fwd_tiles(int Bq, int Bk, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const CUtensorMap& mo, const mala::FwdParams& p, cudaStream_t st) {
+  if (Bq == 128 && Bk == 128) return launch_fwd_gate<D, 128, 128>(gate, mq, mk, mv, mo, p, st);
+  if (Bq == 64 && Bk == 64) return launch_fwd_gate<D, 64, 64>(gate, mq, mk, mv, mo, p, st);
+  if (Bq == 64 && Bk == 128) return launch_fwd_gate<D, 64, 128>(gate, mq, mk, mv, mo, p, st);
+  return launch_fwd_gate<D, 128, 64>(gate, mq, mk, mv, mo, p, st);
 }
 
 // --------------------------------------------------------------- backward
-template <int D, int BK, bool G>
+template <int D, int BQ, int BK, bool G>
 int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                const CUtensorMap& mdk, const CUtensorMap& mdv, const CUtensorMap& mdq, const mala::BwdParams& p,
                cudaStream_t st) {
   using Lay = mala::BwdLayout<D>;
-  auto kern = mala::mala_bwd_kernel<D, BK, G>;
+  auto kern = mala::mala_bwd_kernel<D, BQ, BK, G>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned n_chunks = (p.n_super + p.chunk_kb - 1) / p.chunk_kb;
   const unsigned grid = n_chunks * p.chunk_kb * p.B * p.Hkv;
@@ -156,12 +166,22 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
-template <int D, int BK>
+template <int D, int BQ, int BK>
 int launch_bwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
                     const CUtensorMap& mdq, const mala::BwdParams& p, cudaStream_t st) {
-  return gate ? launch_bwd<D, BK, true>(mq, mk, mv, mdo, mdk, mdv, mdq, p, st)
-              : launch_bwd<D, BK, false>(mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  return gate ? launch_bwd<D, BQ, BK, true>(mq, mk, mv, mdo, mdk, mdv, mdq, p, st)
+              : launch_bwd<D, BQ, BK, false>(mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+}
+
+template <int D>
+int launch_bwd_tiles(int Bq, int Bk, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
+                     const CUtensorMap& mdq, const mala::BwdParams& p, cudaStream_t st) {
+  if (Bq == 128 && Bk == 128) return launch_bwd_gate<D, 128, 128>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  if (Bq == 64 && Bk == 64) return launch_bwd_gate<D, 64, 64>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  if (Bq == 64 && Bk == 128) return launch_bwd_gate<D, 64, 128>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  return launch_bwd_gate<D, 128, 64>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
 }
 
 // ----------------------------------------------------------------- decode
@@ -214,29 +234,30 @@ size_t mala_fwd_workspace_size(int B, int Hkv, int L, int d) {
   return align256(static_cast<size_t>(B) * L * Hkv * d * 2);
 }
 
-int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int L,
-             int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
-             int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
-  if (!q || !k || !v || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
-  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
-  if (rc != MALA_OK) return rc;
+namespace {
+// Forward of Lq queries at positions Lk - Lq .. Lk - 1 against Lk keys (the
+// training forward is Lq == Lk); arguments already checked by the caller.
+int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+            int Lk, int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
+            int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return MALA_ERR_UNSUPPORTED;
-  const size_t need = mala_fwd_workspace_size(B, Hkv, L, d);
+  const size_t need = mala_fwd_workspace_size(B, Hkv, Lk, d);
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap mq, mk, mv, mo;
-  if (!make_bshd_map(&mq, q, B, L, Hq, d, 128) || !make_bshd_map(&mk, k, B, L, Hkv, d, Bk) ||
-      !make_bshd_map(&mv, workspace, B, L, Hkv, d, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_bshd_map(&mo, o, B, L, Hq, d, 128))
+  if (!make_bshd_map(&mq, q, B, Lq, Hq, d, 128) || !make_bshd_map(&mk, k, B, Lk, Hkv, d, Bk) ||
+      !make_bshd_map(&mv, workspace, B, Lk, Hkv, d, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_bshd_map(&mo, o, B, Lq, Hq, d, 128))
     return MALA_ERR_CUDA;
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
   mala::FwdParams p;
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
-  p.nq = (L + Bq - 1) / Bq;
-  p.nk = (L + Bk - 1) / Bk;
-  p.n_pairs = (L + 255) / 256;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+  p.Lq = Lq; p.Lk = Lk; p.P0 = Lk - Lq;
+  p.nq = (Lq + Bq - 1) / Bq;
+  p.nk = (Lk + Bk - 1) / Bk;
+  p.n_pairs = (Lq + 255) / 256;
   p.chunk_pairs = fwd_chunk_pairs(p.n_pairs, p.G);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;
@@ -245,16 +266,36 @@ int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.keep_map = keep_map;
   p.status = status;
   if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
-  const long long n8 = static_cast<long long>(B) * L * Hkv * d / 8;
+  const long long n8 = static_cast<long long>(B) * Lk * Hkv * d / 8;
   const int cv_grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
   mala::mala_v_to_f16_kernel<<<cv_grid, 256, 0, st>>>(static_cast<const uint4*>(v), static_cast<uint4*>(workspace),
                                                       n8, status);
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
   const bool gate = tau > 0.f;
-  if (d == 128 && Bk == 128) return launch_fwd_gate<128, 128>(gate, mq, mk, mv, mo, p, st);
-  if (d == 64 && Bk == 128) return launch_fwd_gate<64, 128>(gate, mq, mk, mv, mo, p, st);
-  if (d == 128 && Bk == 64) return launch_fwd_gate<128, 64>(gate, mq, mk, mv, mo, p, st);
-  return launch_fwd_gate<64, 64>(gate, mq, mk, mv, mo, p, st);
+  if (d == 128) return launch_fwd_tiles<128>(Bq, Bk, gate, mq, mk, mv, mo, p, st);
+  return launch_fwd_tiles<64>(Bq, Bk, gate, mq, mk, mv, mo, p, st);
+}
+}  // namespace
+
+int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int L,
+             int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
+             int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  if (!q || !k || !v || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, L, L, d, scale, tau, Bq, Bk, workspace, workspace_bytes, kept_tiles,
+                 keep_map, stream);
+}
+
+int mala_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                 int Lk, int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
+                 int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  if (!q || !k || !v || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  if (Lq < 1 || Lk < Lq) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(B, Hq, Hkv, Lk, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, tau, Bq, Bk, workspace, workspace_bytes,
+                 kept_tiles, keep_map, stream);
 }
 
 size_t mala_bwd_workspace_size(int B, int Hq, int L, int d) {
@@ -314,10 +355,8 @@ int mala_bwd(const void* q, const void* k, const void* v, const void* o, const v
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
 
   const bool gate = tau > 0.f;
-  if (d == 128 && Bk == 128) rc = launch_bwd_gate<128, 128>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
-  else if (d == 64 && Bk == 128) rc = launch_bwd_gate<64, 128>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
-  else if (d == 128 && Bk == 64) rc = launch_bwd_gate<128, 64>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
-  else rc = launch_bwd_gate<64, 64>(gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  if (d == 128) rc = launch_bwd_tiles<128>(Bq, Bk, gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
+  else rc = launch_bwd_tiles<64>(Bq, Bk, gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
   if (rc != MALA_OK) return rc;
 
   const long long n8 = static_cast<long long>(B) * L * Hq * d / 8;

@@ -79,14 +79,14 @@ struct BwdLayout {
   static_assert(ALLOC_BYTES <= 232448, "backward shared memory exceeds the per-CTA limit");
 };
 
-template <int D, int BK, bool kGate>
+template <int D, int BQ, int BK, bool kGate>
 __global__ void __launch_bounds__(448, 1)
     mala_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Lay = BwdLayout<D>;
-  constexpr int BQ = BK, QPB = 128 / BQ, KPB = 128 / BK;
+  constexpr int QPB = 128 / BQ, KPB = 128 / BK;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
   constexpr uint32_t IDESC_KN = idesc_bf16(128, D, false, true);  // A K-major, B MN-major
   constexpr uint32_t IDESC_MN = idesc_bf16(128, D, true, true);   // A, B MN-major

@@ -11,6 +11,9 @@
 // One CTA owns two 128-row query tiles (A = rows r0..r0+127, B = the next 128)
 // of one (b, hq) and walks key tiles kb = last ... 0. A 128-row tile holds one
 // query block when Bq = 128 and two when Bq = 64; decisions are per block.
+// The same kernel runs prefill against an existing cache: query row r sits at
+// position P0 + r (P0 = Lk - Lq), sees keys 0 .. P0 + r and uses Lq = P0 + r + 1
+// in its threshold; the training forward is P0 = 0, Lq = Lk.
 //   warps 0-3  softmax warpgroup of tile A (thread t = row t = TMEM lane t)
 //   warps 4-7  softmax warpgroup of tile B
 //   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring
@@ -35,8 +38,9 @@
 namespace mala {
 
 struct FwdParams {
-  int B, Hq, Hkv, L, G;
-  int nq, nk, n_pairs;  // n_pairs = ceil(L / 256) pairs of 128-row tiles
+  int B, Hq, Hkv, G;
+  int Lq, Lk, P0;       // Lq queries at positions P0 .. P0 + Lq - 1 of Lk keys (P0 = Lk - Lq)
+  int nq, nk, n_pairs;  // nq = ceil(Lq / Bq), nk = ceil(Lk / Bk), n_pairs = ceil(Lq / 256)
   int chunk_pairs;      // CTA schedule: pairs per chunk (see mala_fwd_kernel)
   float scale_log2;     // scale * log2(e): scores are kept in log2 units
   float log2_tau;       // log2(tau), used only when the gate is on
@@ -86,13 +90,13 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-template <int D, int BK, bool kGate>
+template <int D, int BQ, int BK, bool kGate>
 __global__ void __launch_bounds__(320, 1)
     mala_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
   using Lay = FwdLayout<D, BK>;
-  constexpr int BM = Lay::BM, BQ = BK, QPB = BM / BQ;
+  constexpr int BM = Lay::BM, QPB = BM / BQ;
   constexpr int NK = Lay::NK, NV = Lay::NV;
   constexpr uint32_t IDESC_QK = idesc_bf16(128, BK, false, false);
   constexpr uint32_t IDESC_PV = idesc_f16(128, D, false, true);
@@ -137,8 +141,8 @@ __global__ void __launch_bounds__(320, 1)
   const int b = unit / p.Hkv, hkv = unit % p.Hkv, hq = hkv * p.G + in_chunk % p.G;
   const int bh = b * p.Hq + hq;
   const int r0 = pr * 2 * BM;  // first row of tile A
-  const int last_row = min(r0 + 2 * BM, p.L) - 1;
-  const int kb_hi = last_row / BK;
+  const int last_row = min(r0 + 2 * BM, p.Lq) - 1;  // among the queries
+  const int kb_hi = (p.P0 + last_row) / BK;         // key tile of the pair's last query
   const int T = kb_hi + 1;
 
   if (threadIdx.x == 0) {
@@ -283,12 +287,13 @@ __global__ void __launch_bounds__(320, 1)
     const int wq = warp & 3;            // TMEM lane quarter
     const int row0 = r0 + x * BM;
     const int row = row0 + tid;
-    const bool row_ok = row < p.L;
+    const bool row_ok = row < p.Lq;
+    const int pos = p.P0 + row;  // the query's position: it sees keys 0 .. pos
     const int qi = tid / BQ;
     const int qb = (row0 / BQ) + qi;
     const bool blk_exists = qb < p.nq;
-    const int kbf = blk_exists ? (min((qb + 1) * BQ, p.L) - 1) / BK : -1;
-    const float thr = kGate ? p.log2_tau - lg2_approx(static_cast<float>(row + 1)) : 0.f;
+    const int kbf = blk_exists ? (p.P0 + min((qb + 1) * BQ, p.Lq) - 1) / BK : -1;
+    const float thr = kGate ? p.log2_tau - lg2_approx(static_cast<float>(pos + 1)) : 0.f;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + Lay::COL_S + x * BK + lane_base;
     const uint32_t tO = tmem + Lay::COL_O + x * D + lane_base;
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(320, 1)
       const bool ok = mbar_wait_warp(&s_full[x], t & 1, fs);
       local_abort |= !ok;
       tc_fence_after();
-      const bool diag = kb * BK + BK - 1 > row0;
+      const bool diag = kb * BK + BK - 1 > p.P0 + row0;  // some key of the tile is past some row
       // first pass (row max): all loads of the S row in flight at once, one wait
       float M = -INFINITY;
       {
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(320, 1)
           } else {
 #pragma unroll
             for (int j = 0; j < BK; ++j)
-              if (kb * BK + j <= row) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(sv[j]));
+              if (kb * BK + j <= pos) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(sv[j]));
           }
           M = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         }
@@ -404,8 +409,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                   const int key = kb * BK + ch * 32 + 2 * jj;
-                  const bool l0 = row_ok && key <= row;
-                  const bool l1 = row_ok && key + 1 <= row;
+                  const bool l0 = row_ok && key <= pos;
+                  const bool l1 = row_ok && key + 1 <= pos;
                   // masked entries go through ex2 as -inf (-> 0): no branch around the inline asm
                   const float p0 = ex2_approx(l0 ? fmaf(__uint_as_float(sh[c2 * 32 + 2 * jj]), sl2, -m_use) : -INFINITY);
                   const float p1 =
@@ -456,13 +461,13 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         fence_proxy_async_smem();
-        if (row_ok) p.lse[static_cast<size_t>(bh) * p.L + row] = (m_use + lg2_approx(l)) * 0.69314718055994531f;
+        if (row_ok) p.lse[static_cast<size_t>(bh) * p.Lq + row] = (m_use + lg2_approx(l)) * 0.69314718055994531f;
       }
       const unsigned okall = __ballot_sync(0xffffffffu, okf);
       if (lane == 0) evote[x * 4 + wq] = okall == 0xffffffffu ? 1u : 0u;
       named_bar_sync(1 + x, 128);
       const bool store = (evote[x * 4 + 0] & evote[x * 4 + 1] & evote[x * 4 + 2] & evote[x * 4 + 3]) != 0;
-      if (tid == 0 && store && row0 < p.L) {
+      if (tid == 0 && store && row0 < p.Lq) {
         for (int h = 0; h < D / 64; ++h)
           tma_store_4d(&tm_o, sQ + x * Lay::Q_BYTES + h * (BM * 128), h * 64, hq, row0, b);
         tma_store_commit_and_wait();

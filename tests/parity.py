@@ -30,21 +30,26 @@ def rel_l2(a, b) -> float:
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def legal_mask(L, Bq, Bk):
-    nq, nk = -(-L // Bq), -(-L // Bk)
+def legal_mask(L, Bq, Bk, Lk=None):
+    """Legal tiles of L query rows at positions Lk - L .. Lk - 1 against Lk
+    keys (Lk = L: the training case). Query blocks start at the first row."""
+    Lk = L if Lk is None else Lk
+    P0 = Lk - L
+    nq, nk = -(-L // Bq), -(-Lk // Bk)
     m = np.zeros((nq, nk), dtype=bool)
     for qb in range(nq):
-        m[qb, : (min((qb + 1) * Bq, L) - 1) // Bk + 1] = True
+        m[qb, : (P0 + min((qb + 1) * Bq, L) - 1) // Bk + 1] = True
     return m
 
 
-def compare_fwd_decisions(gpu_keep, ora_keep, ora_margin, L, Bq, Bk, rows=None):
+def compare_fwd_decisions(gpu_keep, ora_keep, ora_margin, L, Bq, Bk, rows=None, Lk=None):
     """Walk every selected (b, hq, qb) chain in visit order (kb descending).
 
     Returns dict(bad, in_margin, cascaded, diverged_blocks, compared).
-    ``rows`` restricts to a list of (b, hq, qb); default all.
+    ``rows`` restricts to a list of (b, hq, qb); default all. ``Lk`` > L: a
+    prefill of L new queries against Lk keys.
     """
-    lm = legal_mask(L, Bq, Bk)
+    lm = legal_mask(L, Bq, Bk, Lk)
     B, H, nq, nk = ora_keep.shape
     if rows is None:
         rows = [(b, h, qb) for b in range(B) for h in range(H) for qb in range(nq)]
@@ -97,8 +102,8 @@ def compare_bwd_decisions(gpu_keep, ora_keep, ora_margin, L, Bq, Bk, diverged_bl
     return out
 
 
-def illegal_untouched(keep_map, L, Bq, Bk) -> bool:
+def illegal_untouched(keep_map, L, Bq, Bk, Lk=None) -> bool:
     """Entries of illegal tiles keep the caller's fill value 255."""
-    lm = legal_mask(L, Bq, Bk)
+    lm = legal_mask(L, Bq, Bk, Lk)
     km = np.asarray(keep_map)
     return bool((km[..., ~lm] == 255).all()) and bool(np.isin(km[..., lm], (0, 1)).all())

@@ -49,11 +49,31 @@ def fwd(**kw):
     (dict(q=None), 1), (dict(lse=None), 1), (dict(kept_tiles=None), 1),
     (dict(B=0), 1), (dict(L=0), 1), (dict(Hq=3, Hkv=2), 1),
     (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(tau=-1.0), 1), (dict(tau=float("inf")), 1),
-    (dict(d=96), 2), (dict(Bq=64, Bk=128), 2), (dict(Bq=32, Bk=32), 2), (dict(q=P + 8), 2),
+    (dict(d=96), 2), (dict(Bq=96, Bk=128), 2), (dict(Bq=128, Bk=256), 2), (dict(Bq=32, Bk=32), 2),
+    (dict(q=P + 8), 2),
     (dict(workspace=None), 3), (dict(workspace_bytes=100), 3), (dict(workspace=P + 16), 3),
 ])
 def test_fwd_rejects(kw, code):
     assert fwd(**kw) == code
+
+
+def pre(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=1, Lq=100, Lk=300, d=128, scale=0.1, tau=1.0, Bq=128,
+             Bk=64, workspace=P, workspace_bytes=1 << 30, kept_tiles=P, keep_map=None, stream=S)
+    a.update(kw)
+    return mala.mala_prefill(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(v=None), 1), (dict(o=None), 1), (dict(kept_tiles=None), 1), (dict(Lq=0), 1), (dict(Lk=99), 1),
+    (dict(Lq=0, Lk=0), 1), (dict(Hq=4, Hkv=3), 1), (dict(tau=float("nan")), 1),
+    (dict(d=256), 2), (dict(Bq=256), 2), (dict(Bk=32), 2), (dict(lse=P + 4), 2),
+    (dict(workspace=None), 3), (dict(workspace=P + 128), 3),
+    # the fp16 V copy covers all Lk keys, not only the new ones
+    (dict(workspace_bytes=(300 * 128 * 2 + 255) // 256 * 256 - 1), 3),
+])
+def test_prefill_rejects(kw, code):
+    assert pre(**kw) == code
 
 
 def bwd(**kw):

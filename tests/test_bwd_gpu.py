@@ -81,7 +81,7 @@ def run_bwd_case(mala, w, tau, L=None, sample=None):
             a = np.concatenate([g[name][b, r, h].ravel() for (b, r, h) in rows_of(selk, w.Bk, L)])
             e = np.concatenate([refb[name][b, r, h].ravel() for (b, r, h) in rows_of(selk, w.Bk, L)])
             errs[name] = rel_l2(a, e)
-    print(f"[bwd parity] L={L} d={d} H={Hq}/{Hkv} B={w.Bq} tau={tau}: "
+    print(f"[bwd parity] L={L} d={d} H={Hq}/{Hkv} Bq={w.Bq} Bk={w.Bk} tau={tau}: "
           + " ".join(f"{n}={v:.3e}" for n, v in errs.items())
           + f" tiles={bd['compared']} in_margin={bd['in_margin']} excused={bd['excused']} kept={int(kb_h.sum())}")
     for name, e in errs.items():
@@ -105,6 +105,18 @@ def test_bwd_c0(cuda_lib, tau):
 ])
 def test_bwd_small_shapes(cuda_lib, L, d, Hq, Hkv, Bt, tau):
     w = TrainWorkload("small", 1, Hq, Hkv, L, d, Bt, Bt, seed=4000 + L + d)
+    run_bwd_case(cuda_lib, w, tau)
+
+
+@pytest.mark.parametrize("L,d,Hq,Hkv,Bq,Bk,tau", [
+    (1000, 128, 4, 2, 64, 128, 1.0),
+    (1000, 128, 4, 2, 128, 64, 1.0),
+    (777, 64, 2, 1, 128, 64, 0.5),
+    (513, 64, 2, 2, 64, 128, 4.0),
+    (700, 128, 2, 1, 64, 128, 0.0),
+])
+def test_bwd_mixed_tiles(cuda_lib, L, d, Hq, Hkv, Bq, Bk, tau):
+    w = TrainWorkload("mixed", 1, Hq, Hkv, L, d, Bq, Bk, seed=4200 + L + Bq)
     run_bwd_case(cuda_lib, w, tau)
 
 

@@ -47,7 +47,7 @@ def run_fwd_case(mala, w, tau, L=None):
     assert e_lse <= LSE_ABS, e_lse
     if tau == 0:
         assert (km_h == 1).sum() == (ref["keep"] == 1).sum()
-    print(f"[fwd parity] L={L} d={w.d} H={w.Hq}/{w.Hkv} B={w.Bq} tau={tau}: o_rel_l2={e_o:.3e} "
+    print(f"[fwd parity] L={L} d={w.d} H={w.Hq}/{w.Hkv} Bq={w.Bq} Bk={w.Bk} tau={tau}: o_rel_l2={e_o:.3e} "
           f"lse_abs={e_lse:.3e} tiles={dec['compared']} in_margin={dec['in_margin']} cascaded={dec['cascaded']} "
           f"kept={int(kept_h.sum())}")
     return {"o_rel_l2": e_o, "lse_abs": e_lse, **{k_: v_ for k_, v_ in dec.items() if k_ != "diverged_blocks"}}
@@ -69,6 +69,18 @@ def test_fwd_c0(cuda_lib, tau):
 ])
 def test_fwd_small_shapes(cuda_lib, L, d, Hq, Hkv, Bt, tau):
     w = TrainWorkload("small", 1, Hq, Hkv, L, d, Bt, Bt, seed=3000 + L + d)
+    run_fwd_case(cuda_lib, w, tau)
+
+
+@pytest.mark.parametrize("L,d,Hq,Hkv,Bq,Bk,tau", [
+    (1000, 128, 4, 2, 64, 128, 1.0),   # two query blocks per key tile, ragged, GQA
+    (1000, 128, 4, 2, 128, 64, 1.0),   # two key blocks per 128 keys
+    (777, 64, 2, 1, 128, 64, 0.5),
+    (513, 64, 2, 2, 64, 128, 4.0),
+    (700, 128, 2, 1, 128, 64, 0.0),
+])
+def test_fwd_mixed_tiles(cuda_lib, L, d, Hq, Hkv, Bq, Bk, tau):
+    w = TrainWorkload("mixed", 1, Hq, Hkv, L, d, Bq, Bk, seed=3200 + L + Bq)
     run_fwd_case(cuda_lib, w, tau)
 
 
