@@ -78,7 +78,11 @@ MALA_API int mala_abi_version(void);
  * row r with a live key satisfies
  *     max_live_j exp(s_rj - m_r) / l_r >= tau / (i_r + 1)      (ties keep).
  * A kept tile updates (m, l) and O for every row of the block; a skipped
- * tile loads no V and does no softmax update and no PV. The PV product runs in
+ * tile does no softmax update and no PV. V tiles are fetched ahead for every
+ * tile, kept or not (they come from L2 and the kernel is not memory-bound;
+ * fetching only after the vote measured slower), so a skip saves the softmax
+ * update and the PV but not the V load; mala_decode keeps the strict rule.
+ * The PV product runs in
  * fp16 on an fp16 copy of V made by the call in `workspace`; V values must lie
  * inside the fp16 range (|v| <= 65504); larger ones are clamped and reported
  * as MALA_ERR_RANGE by mala_check_status.

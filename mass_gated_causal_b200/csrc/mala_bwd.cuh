@@ -430,13 +430,13 @@ __global__ void __launch_bounds__(448, 1)
       }
       bool hit;
       if (kGate) {
-        float m8[8];
+        float m8[8];  // eight independent partial maxima, two columns per step
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sh[e]);
+        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(__uint_as_float(sh[2 * e]), __uint_as_float(sh[2 * e + 1]));
 #pragma unroll
-        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(sh[c]));
-        const float m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int c = 16; c < 64; c += 2)
+          m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], __uint_as_float(sh[c]), __uint_as_float(sh[c + 1]));
+        const float m = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         // max_c(s_c) * sl2 == max_c(s_c * sl2): rounding is monotone
         const float thr = lse2_row + p.log2_tau - lg2_approx(static_cast<float>(qs * 128 + row + 1));
         hit = ok && m * sl2 >= thr;

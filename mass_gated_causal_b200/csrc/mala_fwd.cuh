@@ -6,7 +6,7 @@
 // evolving online-softmax state is compared with tau/Lq (Lq = i + 1); tiles run
 // from the diagonal toward earlier keys; the first legal tile is kept; one
 // row that fails to skip keeps the tile for the whole query block; a skipped
-// tile loads no V and does no softmax update and no PV; LSE is written.
+// tile does no softmax update and no PV; LSE is written.
 //
 // One CTA owns two 128-row query tiles (A = rows r0..r0+127, B = the next 128)
 // of one (b, hq) and walks key tiles kb = last ... 0. A 128-row tile holds one
@@ -16,16 +16,24 @@
 // in its threshold; the training forward is P0 = 0, Lq = Lk.
 //   warps 0-3  softmax warpgroup of tile A (thread t = row t = TMEM lane t)
 //   warps 4-7  softmax warpgroup of tile B
-//   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring
-//              (and, with the gate off, V tiles through the V ring)
+//   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring,
+//              V tiles (fetched or passed over) through an NV ring
 //   warp  9    MMA issuer (one thread)
 // TMEM: S_A | S_B | O_A | O_B. P (fp16) is written over the first half of its
 // tile's S columns and read from TMEM by the PV MMA (A operand in TMEM).
 // The MMA thread alternates between the tiles -- PV_A(t), QK_A(t+1), PV_B(t),
 // QK_B(t+1) -- so the tensor core works on one tile while the other tile's
-// warpgroup runs its gate and softmax. With the gate on, V(t) is requested by
-// TMA only after a warpgroup's vote has kept tile t, so skipped tiles cost no
-// V traffic.
+// warpgroup runs its gate and softmax.
+//
+// V is fetched ahead for every tile, kept or not; a skipped tile gets no
+// softmax update and no PV, and its V tile is never read. The pages list V
+// loads among the work a skip saves; here they are kept on purpose. A CTA's K
+// and V tiles come from L2 (the CTAs of one KV head run together), the kernel
+// is bound by the softmax and the QK -> softmax -> PV chain rather than by
+// memory, and a V load requested only after the vote put its latency on that
+// chain: measured at 32K, GQA 32/8, fetching every V was faster at tau = 1, 4
+// and 16 than fetching V only for kept tiles (or for predicted ones). The
+// memory-bound decode kernel keeps the strict rule.
 //
 // Precision: S = Q K^T is bf16 x bf16 -> fp32. PV runs in fp16 x fp16 -> fp32:
 // P is at most 2^8 (lazy-rescale bound) and V is read from an fp16 copy made
@@ -191,7 +199,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int h = 0; h < D / 64; ++h)
           tma_load_4d(&tm_k, &k_full[st], sK + st * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, kb * BK, b);
         issued = t + 1;
-        if (!kGate) {  // no gate: every V tile is needed, fetch it ahead
+        // V(t) is fetched ahead into slot t % NV whatever the vote decides
+        // (see the note on V above)
+        {
           const int vs = t % NV;
           if (t >= NV && !mbar_wait(&v_empty[vs], ((t / NV) - 1) & 1, fs)) break;
           mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
@@ -212,7 +222,6 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dVm = sdesc_sw128(smem_u32(sV), BK * 128, 1024);
-      int nv = 0;  // V loads issued (gate on)
       int npv[2] = {0, 0};
       auto issue_qk = [&](int x, int t) {
         const int st = t % NK;
@@ -242,26 +251,15 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(&k_empty[0]);
       }
       for (int t = 0; ok && t < T; ++t) {
-        const int kb = kb_hi - t;
-        int vslot = kGate ? -1 : t % NV;
+        const int vslot = t % NV;
         for (int x = 0; x < 2 && ok; ++x) {
           if (!mbar_wait(&dec_bar[x], t & 1, fs)) { ok = false; break; }
           const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&dec_flags[x]);
           if (dec & kDecAbort) { ok = false; break; }
           const bool keep = (dec & kDecPV) != 0;
-          if (kGate && keep && vslot < 0) {  // the vote kept tile t: only now request V(t)
-            vslot = nv % NV;
-            if (nv >= NV && !mbar_wait(&v_empty[vslot], ((nv / NV) - 1) & 1, fs)) { ok = false; break; }
-            mbar_arrive_expect_tx(&v_full[vslot], Lay::KV_BYTES);
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_4d(&tm_v, &v_full[vslot], sV + vslot * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv,
-                          kb * BK, b);
-            ++nv;
-          }
           if (!mbar_wait(&sm_done[x], t & 1, fs)) { ok = false; break; }  // P_x(t) written (or S_x released)
           if (keep) {
-            const int vi = kGate ? nv - 1 : t;
-            if (!mbar_wait(&v_full[vslot], (vi / NV) & 1, fs)) { ok = false; break; }
+            if (!mbar_wait(&v_full[vslot], (t / NV) & 1, fs)) { ok = false; break; }
             tc_fence_after();
             issue_pv(x, vslot);
           }
@@ -273,11 +271,9 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (!ok) break;
-        if (vslot >= 0) umma_commit(&v_empty[vslot]);  // V(t) has been read by both PVs
+        umma_commit(&v_empty[vslot]);  // V(t) read by both PVs (or not needed)
       }
       umma_commit(mma_final);  // completes once every MMA above has finished
-      if (kGate)
-        for (int i = max(0, nv - NV); i < nv; ++i) mbar_wait_drain(&v_full[i % NV], (i / NV) & 1);
     }
     __syncwarp();
   } else {
@@ -318,18 +314,20 @@ __global__ void __launch_bounds__(320, 1)
         for (int ch = 0; ch < BK / 32; ++ch) tmem_ld32_at(tS + ch * 32, sv + ch * 32);
         tmem_ld_wait();
         if (ok) {
-          float mp[8];  // eight independent partial maxima (short dependency chains)
+          float mp[8];  // eight independent partial maxima (short dependency chains), two columns per step
 #pragma unroll
           for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
           if (!diag) {
 #pragma unroll
-            for (int j = 0; j < BK; ++j) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(sv[j]));
+            for (int j = 0; j < BK; j += 2)
+              mp[(j >> 1) & 7] = fmax3(mp[(j >> 1) & 7], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
           } else {
 #pragma unroll
-            for (int j = 0; j < BK; ++j)
-              if (kb * BK + j <= pos) mp[j & 7] = fmaxf(mp[j & 7], __uint_as_float(sv[j]));
+            for (int j = 0; j < BK; j += 2)
+              mp[(j >> 1) & 7] = fmax3(mp[(j >> 1) & 7], kb * BK + j <= pos ? __uint_as_float(sv[j]) : -INFINITY,
+                                       kb * BK + j + 1 <= pos ? __uint_as_float(sv[j + 1]) : -INFINITY);
           }
-          M = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+          M = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
         }
       }
       const bool legal = blk_exists && kb <= kbf;
