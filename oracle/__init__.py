@@ -224,3 +224,144 @@ def decode(q, kc, vc, scale: float, tau: float, Bk: int, n_splits: int,
     if with_parts:
         out["o_part"], out["lse_part"] = op, lp
     return out
+
+
+# ------------------------------------------------------------------ packed batches
+# A packed (variable-length) batch is a set of independent sequences laid end to
+# end; MALA's gate never looks across a sequence. These functions are that
+# definition written out: each sequence's slice goes through the single-sequence
+# routines above, whose arithmetic is pinned on its own.
+
+def _cu(cu):
+    cu = np.asarray(cu, dtype=np.int64)
+    assert cu.ndim == 1 and cu[0] == 0 and (np.diff(cu) >= 0).all()
+    return cu
+
+
+def varlen_fwd(q, k, v, cu_q, cu_k, scale: float, tau: float, Bq: int, Bk: int, with_margin: bool = True):
+    """MALA forward of a packed batch. q [total_q,Hq,d]; k/v [total_k,Hkv,d];
+    sequence s owns query rows cu_q[s]:cu_q[s+1] and keys cu_k[s]:cu_k[s+1]
+    (Lk_s >= Lq_s: its queries are the last Lq_s of its Lk_s positions, as in
+    ``prefill``; Lq_s == Lk_s is the training forward).
+
+    Returns dict with o [total_q,Hq,d], lse [Hq,total_q], keep / margin
+    [S,Hq,max_nq,max_nk] (per sequence its [nq_s, nk_s] corner; legal entries
+    0/1, the rest 255 / NaN) and kept [S*Hq].
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu_q, cu_k = _cu(cu_q), _cu(cu_k)
+    S = len(cu_q) - 1
+    assert len(cu_k) == S + 1
+    Hq, d = q.shape[1], q.shape[2]
+    lq, lk = np.diff(cu_q), np.diff(cu_k)
+    assert (lk >= lq).all()
+    mq = max(1, -(-int(lq.max(initial=0)) // Bq))
+    mk = max(1, -(-int(lk.max(initial=0)) // Bk))
+    o = np.full_like(q, np.nan)
+    lse = np.full((Hq, q.shape[0]), np.nan)
+    keep = np.full((S, Hq, mq, mk), 255, dtype=np.uint8)
+    margin = np.full((S, Hq, mq, mk), np.nan) if with_margin else None
+    kept = np.zeros(S * Hq, dtype=np.int64)
+    for s in range(S):
+        if lq[s] == 0:
+            continue
+        r = prefill(q[None, cu_q[s]:cu_q[s + 1]], k[None, cu_k[s]:cu_k[s + 1]], v[None, cu_k[s]:cu_k[s + 1]],
+                    scale, tau, Bq, Bk, with_margin=with_margin)
+        o[cu_q[s]:cu_q[s + 1]] = r["o"][0]
+        lse[:, cu_q[s]:cu_q[s + 1]] = r["lse"][0]
+        nq_s, nk_s = r["keep"].shape[2], r["keep"].shape[3]
+        legal = _legal(int(lq[s]), int(lk[s]), Bq, Bk)
+        blk = keep[s, :, :nq_s, :nk_s]
+        blk[:, legal] = r["keep"][0][:, legal]
+        if with_margin:
+            margin[s, :, :nq_s, :nk_s] = r["margin"][0]
+        kept[s * Hq:(s + 1) * Hq] = r["kept"]
+    return {"o": o, "lse": lse, "keep": keep, "margin": margin, "kept": kept}
+
+
+def _legal(Lq: int, Lk: int, Bq: int, Bk: int):
+    """[nq, nk] legal-tile mask of Lq queries at positions Lk-Lq.. against Lk keys."""
+    P0 = Lk - Lq
+    nq, nk = -(-Lq // Bq), -(-Lk // Bk)
+    m = np.zeros((nq, nk), dtype=bool)
+    for qb in range(nq):
+        m[qb, : (P0 + min((qb + 1) * Bq, Lq) - 1) // Bk + 1] = True
+    return m
+
+
+def varlen_bwd(q, k, v, o, do, lse, cu, scale: float, tau: float, Bq: int, Bk: int, with_margin: bool = True):
+    """MALA backward of a packed training batch (queries and keys share ``cu``).
+    q/o/do [total,Hq,d], k/v [total,Hkv,d], lse [Hq,total] (as ``varlen_fwd``
+    returns it). Returns dq, dk, dv (packed like the inputs), keep / margin
+    [S,Hq,max_nq,max_nk] (illegal entries 255 / NaN) and kept [S*Hq]."""
+    q, k, v, o, do, lse = (_f64(a) for a in (q, k, v, o, do, lse))
+    cu = _cu(cu)
+    S = len(cu) - 1
+    Hq = q.shape[1]
+    ln = np.diff(cu)
+    mq = max(1, -(-int(ln.max(initial=0)) // Bq))
+    mk = max(1, -(-int(ln.max(initial=0)) // Bk))
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    keep = np.full((S, Hq, mq, mk), 255, dtype=np.uint8)
+    margin = np.full((S, Hq, mq, mk), np.nan) if with_margin else None
+    kept = np.zeros(S * Hq, dtype=np.int64)
+    for s in range(S):
+        a, b = cu[s], cu[s + 1]
+        if b == a:
+            continue
+        r = bwd(q[None, a:b], k[None, a:b], v[None, a:b], o[None, a:b], do[None, a:b], lse[None, :, a:b],
+                scale, tau, Bq, Bk, with_margin=with_margin)
+        dq[a:b], dk[a:b], dv[a:b] = r["dq"][0], r["dk"][0], r["dv"][0]
+        legal = _legal(int(b - a), int(b - a), Bq, Bk)
+        nq_s, nk_s = legal.shape
+        blk = keep[s, :, :nq_s, :nk_s]
+        blk[:, legal] = r["keep"][0][:, legal]
+        if with_margin:
+            margin[s, :, :nq_s, :nk_s] = r["margin"][0]
+        kept[s * Hq:(s + 1) * Hq] = r["kept"]
+    return {"dq": dq, "dk": dk, "dv": dv, "keep": keep, "margin": margin, "kept": kept}
+
+
+def paged_decode(q, k_pages, v_pages, block_table, seqlens, scale: float, tau: float, n_splits: int,
+                 sel: Optional[Sequence] = None):
+    """MALA decode against a paged KV cache. q [B,Hq,d]; k_pages/v_pages
+    [num_pages,page,Hkv,d]; block_table [B,max_pages] (page ids); seqlens [B].
+    Sequence b's keys are rows 0..page-1 of pages block_table[b,0], [b,1], ...,
+    cut at seqlens[b]; its key tiles are its pages (Bk = page). Each sequence is
+    ``decode`` of its gathered cache with the same n_splits.
+
+    Returns dict with o [B,Hq,d], lse [B,Hq], keep / margin [B,Hq,max_pages]
+    (entries past a sequence's tiles 255 / NaN), kept [B*Hq]. ``sel`` lists
+    (b, hq) rows to compute; other rows are NaN (keep 255)."""
+    q, kp, vp = _f64(q), _f64(k_pages), _f64(v_pages)
+    bt = np.asarray(block_table, dtype=np.int64)
+    sl = np.asarray(seqlens, dtype=np.int64)
+    B, Hq, d = q.shape
+    page = kp.shape[1]
+    maxp = bt.shape[1]
+    o = np.full((B, Hq, d), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    keep = np.full((B, Hq, maxp), 255, dtype=np.uint8)
+    margin = np.full((B, Hq, maxp), np.nan)
+    kept = np.zeros(B * Hq, dtype=np.int64)
+    rows = None if sel is None else {}
+    if sel is not None:
+        for (b, hq) in sel:
+            rows.setdefault(int(b), []).append(int(hq))
+    for b in range(B):
+        if rows is not None and b not in rows:
+            continue
+        Lk = int(sl[b])
+        npg = -(-Lk // page)
+        kc = kp[bt[b, :npg]].reshape(npg * page, kp.shape[2], d)[:Lk]
+        vc = vp[bt[b, :npg]].reshape(npg * page, vp.shape[2], d)[:Lk]
+        s = None if rows is None else [(0, hq) for hq in sorted(set(rows[b]))]
+        r = decode(q[b:b + 1], kc[None], vc[None], scale, tau, page, n_splits, sel=s)
+        hs = range(Hq) if rows is None else sorted(set(rows[b]))
+        for hq in hs:
+            o[b, hq] = r["o"][0, hq]
+            lse[b, hq] = r["lse"][0, hq]
+            keep[b, hq, :npg] = r["keep"][0, hq]
+            margin[b, hq, :npg] = r["margin"][0, hq]
+            kept[b * Hq + hq] = r["kept"][hq]
+    return {"o": o, "lse": lse, "keep": keep, "margin": margin, "kept": kept}
