@@ -50,7 +50,8 @@ extern "C" {
 
 typedef enum mala_status {
     MALA_OK = 0,
-    MALA_ERR_INVALID_ARG = 1,    /* null pointer, Hq % Hkv != 0, L < 1, scale <= 0, tau < 0, NaN */
+    MALA_ERR_INVALID_ARG = 1,    /* null pointer, Hq % Hkv != 0, L < 1, scale <= 0, tau < 0, NaN;
+                                    also a bad device-side sequence or page table (mala_check_status) */
     MALA_ERR_UNSUPPORTED = 2,    /* d, Bq, Bk outside the supported set; pointer not 16-B aligned */
     MALA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than the size query returns */
     MALA_ERR_CUDA = 4,           /* a CUDA runtime / driver call or a launch failed */
@@ -142,6 +143,39 @@ MALA_API int mala_prefill(const void* q, const void* k, const void* v, void* o, 
              size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
 
 /*
+ * mala_fwd_varlen -- MALA forward of a packed batch of variable-length
+ * sequences (training, or prefill of several prompts against their caches).
+ *
+ * Source: as mala_fwd / mala_prefill; a packed batch is independent sequences
+ * laid end to end (the gate never looks across a sequence).
+ *
+ * Sequence s (0 <= s < num_seqs) owns query rows cu_seqlens_q[s] ..
+ * cu_seqlens_q[s+1] - 1 of q / o and key rows cu_seqlens_k[s] ..
+ * cu_seqlens_k[s+1] - 1 of k / v; with Lq_s and Lk_s its lengths (Lk_s >= Lq_s,
+ * Lq_s may be 0) it is exactly mala_prefill(Lq = Lq_s, Lk = Lk_s).
+ *
+ *   q, o       [total_q, Hq, d]  bf16 (in / out)
+ *   k, v       [total_k, Hkv, d] bf16, in
+ *   lse        [Hq, total_q]     fp32, out (natural log)
+ *   cu_seqlens_q, cu_seqlens_k  [num_seqs + 1] int32, DEVICE memory, in:
+ *              non-decreasing offsets starting at 0, ending at total_q / total_k
+ *   max_seqlen_q, max_seqlen_k  bounds on Lq_s and Lk_s (they size the grid and keep_map)
+ *   workspace  >= mala_fwd_workspace_size(1, Hkv, total_k, d) bytes
+ *   kept_tiles [num_seqs * Hq] int32, out (required)
+ *   keep_map   [num_seqs, Hq, ceil(max_seqlen_q / Bq), ceil(max_seqlen_k / Bk)] uint8,
+ *              nullable; per sequence its legal tiles are written, the rest untouched
+ * The sequence tables live on the device and are checked there: a sequence
+ * whose entries are out of range (offsets outside the tensors, Lk_s < Lq_s, or
+ * a length above the stated maximum) is left untouched and mala_check_status
+ * returns MALA_ERR_INVALID_ARG.
+ */
+MALA_API int mala_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int num_seqs, int max_seqlen_q,
+             int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale, float tau,
+             int Bq, int Bk, void* workspace, size_t workspace_bytes, int32_t* kept_tiles,
+             uint8_t* keep_map, void* stream);
+
+/*
  * Workspace bytes mala_bwd needs: an fp32 dQ accumulator [B, L, Hq, d] and
  * an fp32 D = rowsum(dO * O) vector [B, Hq, L], each 256-byte aligned.
  * Returns 0 for invalid sizes.
@@ -177,6 +211,26 @@ MALA_API int mala_bwd(const void* q, const void* k, const void* v, const void* o
              const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int L, int d,
              float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
              int32_t* kept_tiles, uint8_t* keep_map, void* stream);
+
+/*
+ * mala_bwd_varlen -- MALA backward of a packed training batch (the queries and
+ * keys of sequence s are rows cu_seqlens[s] .. cu_seqlens[s+1] - 1).
+ *
+ * Source: as mala_bwd, per sequence.
+ *
+ *   q, o, dO, dq  [total, Hq, d]  bf16; k, v, dk, dv [total, Hkv, d] bf16
+ *   lse           [Hq, total] fp32, as mala_fwd_varlen writes it
+ *   cu_seqlens    [num_seqs + 1] int32, DEVICE memory; max_seqlen bounds every length
+ *   workspace     >= mala_bwd_workspace_size(1, Hq, total, d) bytes
+ *   kept_tiles    [num_seqs * Hq] int32, out; keep_map [num_seqs, Hq,
+ *                 ceil(max_seqlen / Bq), ceil(max_seqlen / Bk)] uint8, nullable
+ * Invalid sequence entries are handled as in mala_fwd_varlen.
+ */
+MALA_API int mala_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, void* dq, void* dk, void* dv, const int32_t* cu_seqlens, int num_seqs,
+             int max_seqlen, int total, int Hq, int Hkv, int d, float scale, float tau, int Bq, int Bk,
+             void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
+             void* stream);
 
 /*
  * Workspace bytes mala_decode needs for n_splits partial results:
@@ -221,6 +275,36 @@ MALA_API int mala_decode(const void* q, const void* kcache, const void* vcache, 
                 int Hq, int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits,
                 void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
                 void* stream);
+
+/*
+ * mala_decode_paged -- mala_decode against a paged KV cache.
+ *
+ * Source: as mala_decode (the cache is kept whole; decode reads it).
+ *
+ * The keys of sequence b are rows 0 .. page_size - 1 of pages
+ * block_table[b * max_pages_per_seq + 0], [.. + 1], ... of the page pools, cut
+ * at seqlens_k[b] (1 <= seqlens_k[b] <= max_pages_per_seq * page_size). A page
+ * is one key tile (Bk = page_size). Each sequence is split into n_splits
+ * contiguous ranges of ceil(nk_b / n_splits) tiles (nk_b = its page count), so
+ * results equal mala_decode of the gathered cache with the same n_splits.
+ *
+ *   q          [B, Hq, d] bf16, in;  o [B, Hq, d] bf16, out;  lse [B, Hq] fp32, out
+ *   k_pages, v_pages  [num_pages, page_size, Hkv, d] bf16, in
+ *   block_table [B, max_pages_per_seq] int32, DEVICE memory (entries past a
+ *              sequence's pages are not read)
+ *   seqlens_k  [B] int32, DEVICE memory
+ *   page_size  64 or 128;  n_splits >= 1, or 0 for
+ *              mala_decode_default_splits(B, Hkv, max_pages_per_seq * page_size, page_size)
+ *   workspace  >= mala_decode_workspace_size(B, Hq, d, n_splits used) bytes
+ *   kept_tiles [B*Hq] int32, out; keep_map [B, Hq, max_pages_per_seq] uint8, nullable
+ * A length out of range or a page id outside [0, num_pages) is reported by
+ * mala_check_status as MALA_ERR_INVALID_ARG (such a page reads as zeros).
+ */
+MALA_API int mala_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+             const int32_t* block_table, const int32_t* seqlens_k, void* o, float* lse, int B, int Hq,
+             int Hkv, int num_pages, int page_size, int max_pages_per_seq, int d, float scale, float tau,
+             int n_splits, void* workspace, size_t workspace_bytes, int32_t* kept_tiles,
+             uint8_t* keep_map, void* stream);
 
 /*
  * mala_decode_noalloc -- mala_decode without a caller-provided workspace.

@@ -5,9 +5,11 @@ this module only turns torch tensors into device pointers, allocates outputs
 with torch and passes the current CUDA stream. There is no CPU fallback: if the
 library is missing, importing this package raises.
 
-Raw entry points keep the C names (``mala_fwd``, ``mala_prefill``, ``mala_bwd``,
-``mala_decode``, ...). ``forward``, ``prefill``, ``backward`` and ``decode`` are
-conveniences that allocate the outputs and workspaces.
+Raw entry points keep the C names (``mala_fwd``, ``mala_prefill``, ``mala_fwd_varlen``,
+``mala_bwd``, ``mala_bwd_varlen``, ``mala_decode``, ``mala_decode_paged``, ...).
+``forward``, ``prefill``, ``forward_varlen``, ``backward``, ``backward_varlen``,
+``decode`` and ``decode_paged`` are conveniences that allocate the outputs and
+workspaces.
 """
 from __future__ import annotations
 
@@ -33,11 +35,10 @@ MALA_ERR_CUDA = 4
 MALA_ERR_DEVICE_TIMEOUT = 5
 MALA_ERR_RANGE = 6
 
-EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_prefill", "mala_fwd_workspace_size",
-            "mala_bwd_workspace_size",
-            "mala_bwd",
-            "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_noalloc_max_bytes",
-            "mala_decode_noalloc", "mala_check_status")
+EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_prefill", "mala_fwd_varlen",
+            "mala_fwd_workspace_size", "mala_bwd_workspace_size", "mala_bwd", "mala_bwd_varlen",
+            "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_paged",
+            "mala_decode_noalloc_max_bytes", "mala_decode_noalloc", "mala_check_status")
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _lib.mala_status_string.argtypes = [_i]
@@ -48,6 +49,15 @@ _lib.mala_fwd.restype = _i
 _lib.mala_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp,
                               _vp]
 _lib.mala_prefill.restype = _i
+_lib.mala_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _f, _i, _i,
+                                 _vp, _sz, _vp, _vp, _vp]
+_lib.mala_fwd_varlen.restype = _i
+_lib.mala_bwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f,
+                                 _i, _i, _vp, _sz, _vp, _vp, _vp]
+_lib.mala_bwd_varlen.restype = _i
+_lib.mala_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _i, _vp,
+                                   _sz, _vp, _vp, _vp]
+_lib.mala_decode_paged.restype = _i
 _lib.mala_fwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.mala_fwd_workspace_size.restype = _sz
 _lib.mala_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
@@ -119,6 +129,32 @@ def mala_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, tau, Bq, Bk, wor
     return int(_lib.mala_prefill(_p(q), _p(k), _p(v), _p(o), _p(lse), B, Hq, Hkv, Lq, Lk, d, float(scale),
                                  float(tau), Bq, Bk, _p(workspace), int(workspace_bytes), _p(kept_tiles),
                                  _p(keep_map), _stream(stream)))
+
+
+def mala_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
+                    total_k, Hq, Hkv, d, scale, tau, Bq, Bk, workspace, workspace_bytes, kept_tiles, keep_map=None,
+                    stream=None) -> int:
+    return int(_lib.mala_fwd_varlen(_p(q), _p(k), _p(v), _p(o), _p(lse), _p(cu_seqlens_q), _p(cu_seqlens_k),
+                                    num_seqs, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d,
+                                    float(scale), float(tau), Bq, Bk, _p(workspace), int(workspace_bytes),
+                                    _p(kept_tiles), _p(keep_map), _stream(stream)))
+
+
+def mala_bwd_varlen(q, k, v, o, do, lse, dq, dk, dv, cu_seqlens, num_seqs, max_seqlen, total, Hq, Hkv, d, scale,
+                    tau, Bq, Bk, workspace, workspace_bytes, kept_tiles, keep_map=None, stream=None) -> int:
+    return int(_lib.mala_bwd_varlen(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), _p(dq), _p(dk), _p(dv),
+                                    _p(cu_seqlens), num_seqs, max_seqlen, total, Hq, Hkv, d, float(scale),
+                                    float(tau), Bq, Bk, _p(workspace), int(workspace_bytes), _p(kept_tiles),
+                                    _p(keep_map), _stream(stream)))
+
+
+def mala_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o, lse, B, Hq, Hkv, num_pages, page_size,
+                      max_pages_per_seq, d, scale, tau, n_splits, workspace, workspace_bytes, kept_tiles,
+                      keep_map=None, stream=None) -> int:
+    return int(_lib.mala_decode_paged(_p(q), _p(k_pages), _p(v_pages), _p(block_table), _p(seqlens_k), _p(o),
+                                      _p(lse), B, Hq, Hkv, num_pages, page_size, max_pages_per_seq, d,
+                                      float(scale), float(tau), n_splits, _p(workspace), int(workspace_bytes),
+                                      _p(kept_tiles), _p(keep_map), _stream(stream)))
 
 
 def mala_fwd_workspace_size(B, Hkv, L, d) -> int:
@@ -207,6 +243,51 @@ def prefill(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, kee
     return o, lse, kept, km
 
 
+def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, scale: float,
+                   tau: float, Bq: int = 128, Bk: int = 128, keep_map: bool = False, workspace=None, stream=None):
+    """Packed batch: q [total_q,Hq,d], k/v [total_k,Hkv,d] bf16; cu_seqlens_* int32 CUDA tensors
+    [num_seqs+1] -> (o [total_q,Hq,d], lse [Hq,total_q], kept_tiles [num_seqs*Hq], keep_map|None)."""
+    import torch
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    S = cu_seqlens_q.numel() - 1
+    if workspace is None:
+        workspace = torch.empty((max(1, mala_fwd_workspace_size(1, Hkv, total_k, d)),), dtype=torch.uint8,
+                                device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    kept = torch.empty((S * Hq,), dtype=torch.int32, device=q.device)
+    km = None
+    if keep_map:
+        km = torch.full((S, Hq, -(-max_seqlen_q // Bq), -(-max_seqlen_k // Bk)), 255, dtype=torch.uint8,
+                        device=q.device)
+    _check(mala_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, S, max_seqlen_q, max_seqlen_k, total_q,
+                           total_k, Hq, Hkv, d, scale, tau, Bq, Bk, workspace,
+                           workspace.numel() * workspace.element_size(), kept, km, stream), "mala_fwd_varlen")
+    return o, lse, kept, km
+
+
+def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int, scale: float, tau: float, Bq: int = 128,
+                    Bk: int = 128, keep_map: bool = False, workspace=None, stream=None):
+    """Packed training batch -> (dq, dk, dv, kept_tiles [num_seqs*Hq], keep_map|None)."""
+    import torch
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    S = cu_seqlens.numel() - 1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    kept = torch.empty((S * Hq,), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty((mala_bwd_workspace_size(1, Hq, total, d),), dtype=torch.uint8, device=q.device)
+    km = None
+    if keep_map:
+        km = torch.full((S, Hq, -(-max_seqlen // Bq), -(-max_seqlen // Bk)), 255, dtype=torch.uint8,
+                        device=q.device)
+    _check(mala_bwd_varlen(q, k, v, o, do, lse, dq, dk, dv, cu_seqlens, S, max_seqlen, total, Hq, Hkv, d, scale,
+                           tau, Bq, Bk, workspace, workspace.numel() * workspace.element_size(), kept, km,
+                           stream), "mala_bwd_varlen")
+    return dq, dk, dv, kept, km
+
+
 def backward(q, k, v, o, do, lse, scale: float, tau: float, Bq: int = 128, Bk: int = 128,
              keep_map: bool = False, workspace=None, stream=None):
     """-> (dq, dk, dv, kept_tiles, keep_map|None)."""
@@ -245,4 +326,27 @@ def decode(q, kcache, vcache, scale: float, tau: float, Bk: int = 128, n_splits:
     km = torch.full((B, Hq, -(-Lk // Bk)), 255, dtype=torch.uint8, device=q.device) if keep_map else None
     _check(mala_decode(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, workspace,
                        workspace.numel() * workspace.element_size(), kept, km, stream), "mala_decode")
+    return o, lse, kept, km, n_splits
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens_k, scale: float, tau: float, n_splits: int = 0,
+                 keep_map: bool = False, workspace=None, stream=None):
+    """q [B,Hq,d]; k_pages/v_pages [num_pages,page,Hkv,d]; block_table [B,max_pages] and
+    seqlens_k [B] int32 CUDA tensors -> (o, lse, kept_tiles, keep_map|None, n_splits)."""
+    import torch
+    B, Hq, d = q.shape
+    num_pages, page, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    maxp = block_table.shape[1]
+    if n_splits == 0:
+        n_splits = mala_decode_default_splits(B, Hkv, maxp * page, page)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    kept = torch.empty((B * Hq,), dtype=torch.int32, device=q.device)
+    ws_bytes = mala_decode_workspace_size(B, Hq, d, n_splits)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=q.device)
+    km = torch.full((B, Hq, maxp), 255, dtype=torch.uint8, device=q.device) if keep_map else None
+    _check(mala_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o, lse, B, Hq, Hkv, num_pages, page, maxp,
+                             d, scale, tau, n_splits, workspace, workspace.numel() * workspace.element_size(), kept,
+                             km, stream), "mala_decode_paged")
     return o, lse, kept, km, n_splits

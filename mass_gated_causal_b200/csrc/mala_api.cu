@@ -158,7 +158,7 @@ int launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
                const CUtensorMap& mdk, const CUtensorMap& mdv, const CUtensorMap& mdq, const mala::BwdParams& p,
                cudaStream_t st) {
   using Lay = mala::BwdLayout<D>;
-  auto kern = mala::mala_bwd_kernel<D, BQ, BK, G>;
+  auto kern = p.cu != nullptr ? mala::mala_bwd_kernel<D, BQ, BK, G, true> : mala::mala_bwd_kernel<D, BQ, BK, G, false>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned n_chunks = (p.n_super + p.chunk_kb - 1) / p.chunk_kb;
   const unsigned grid = n_chunks * p.chunk_kb * p.B * p.Hkv;
@@ -188,7 +188,8 @@ int launch_bwd_tiles(int Bq, int Bk, bool gate, const CUtensorMap& mq, const CUt
 template <int D, int BK, int GP, bool G>
 int launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const mala::DecParams& p, cudaStream_t st) {
   using Lay = mala::DecLayout<D, BK, GP>;
-  auto kern = mala::mala_decode_split_kernel<D, BK, GP, G>;
+  auto kern = p.block_table != nullptr ? mala::mala_decode_split_kernel<D, BK, GP, G, true>
+                                       : mala::mala_decode_split_kernel<D, BK, GP, G, false>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hkv * p.n_splits;
   kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mk, mv, p);
@@ -235,26 +236,42 @@ size_t mala_fwd_workspace_size(int B, int Hkv, int L, int d) {
 }
 
 namespace {
+// Packed batch: sequence tables and sizes (null cu_q for a dense batch).
+struct Packed {
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
+};
+
 // Forward of Lq queries at positions Lk - Lq .. Lk - 1 against Lk keys (the
-// training forward is Lq == Lk); arguments already checked by the caller.
+// training forward is Lq == Lk); arguments already checked by the caller. For a
+// packed batch, B counts the sequences and Lq / Lk are the longest lengths.
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
             int Lk, int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
-            int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+            int32_t* kept_tiles, uint8_t* keep_map, void* stream, const Packed& pk = Packed()) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return MALA_ERR_UNSUPPORTED;
-  const size_t need = mala_fwd_workspace_size(B, Hkv, Lk, d);
+  const bool packed = pk.cu_q != nullptr;
+  // tensor extents: [B, L, H, d], a packed batch as one sequence of all its rows
+  const int tb = packed ? 1 : B, tq = packed ? pk.total_q : Lq, tk = packed ? pk.total_k : Lk;
+  const size_t need = mala_fwd_workspace_size(tb, Hkv, tk, d);
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap mq, mk, mv, mo;
-  if (!make_bshd_map(&mq, q, B, Lq, Hq, d, 128) || !make_bshd_map(&mk, k, B, Lk, Hkv, d, Bk) ||
-      !make_bshd_map(&mv, workspace, B, Lk, Hkv, d, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_bshd_map(&mo, o, B, Lq, Hq, d, 128))
+  if (!make_bshd_map(&mq, q, tb, tq, Hq, d, 128) || !make_bshd_map(&mk, k, tb, tk, Hkv, d, Bk) ||
+      !make_bshd_map(&mv, workspace, tb, tk, Hkv, d, Bk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_bshd_map(&mo, o, tb, tq, Hq, d, 128))
     return MALA_ERR_CUDA;
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
   mala::FwdParams p;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
   p.Lq = Lq; p.Lk = Lk; p.P0 = Lk - Lq;
+  p.o = static_cast<uint16_t*>(o);
+  p.cu_q = pk.cu_q;
+  p.cu_k = pk.cu_k;
+  p.total_q = pk.total_q;
+  p.total_k = pk.total_k;
   p.nq = (Lq + Bq - 1) / Bq;
   p.nk = (Lk + Bk - 1) / Bk;
   p.n_pairs = (Lq + 255) / 256;
@@ -266,7 +283,7 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   p.keep_map = keep_map;
   p.status = status;
   if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
-  const long long n8 = static_cast<long long>(B) * Lk * Hkv * d / 8;
+  const long long n8 = static_cast<long long>(tb) * tk * Hkv * d / 8;
   const int cv_grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
   mala::mala_v_to_f16_kernel<<<cv_grid, 256, 0, st>>>(static_cast<const uint4*>(v), static_cast<uint4*>(workspace),
                                                       n8, status);
@@ -298,36 +315,58 @@ int mala_prefill(const void* q, const void* k, const void* v, void* o, float* ls
                  kept_tiles, keep_map, stream);
 }
 
+int mala_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q,
+                    int total_k, int Hq, int Hkv, int d, float scale, float tau, int Bq, int Bk, void* workspace,
+                    size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  if (!q || !k || !v || !o || !lse || !kept_tiles || !cu_seqlens_q || !cu_seqlens_k) return MALA_ERR_INVALID_ARG;
+  if (num_seqs < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || total_q < 1 || total_k < 1)
+    return MALA_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(1, Hq, Hkv, std::max(total_q, total_k), d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  if (static_cast<long long>(num_seqs) * Hq >= (1ll << 24)) return MALA_ERR_UNSUPPORTED;
+  Packed pk;
+  pk.cu_q = cu_seqlens_q;
+  pk.cu_k = cu_seqlens_k;
+  pk.total_q = total_q;
+  pk.total_k = total_k;
+  return run_fwd(q, k, v, o, lse, num_seqs, Hq, Hkv, max_seqlen_q, max_seqlen_k, d, scale, tau, Bq, Bk, workspace,
+                 workspace_bytes, kept_tiles, keep_map, stream, pk);
+}
+
 size_t mala_bwd_workspace_size(int B, int Hq, int L, int d) {
   if (B < 1 || Hq < 1 || L < 1 || (d != 64 && d != 128)) return 0;
   return align256(static_cast<size_t>(B) * L * Hq * d * 4) + align256(static_cast<size_t>(B) * Hq * L * 4);
 }
 
-int mala_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int L, int d, float scale, float tau, int Bq,
-             int Bk, void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
-             void* stream) {
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !kept_tiles) return MALA_ERR_INVALID_ARG;
-  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
-  if (rc != MALA_OK) return rc;
+namespace {
+// Backward; arguments already checked by the caller. For a packed batch, B
+// counts the sequences and L is the longest length.
+int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+            void* dk, void* dv, int B, int Hq, int Hkv, int L, int d, float scale, float tau, int Bq, int Bk,
+            void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream,
+            const Packed& pk = Packed()) {
   const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
   for (const void* x : ptrs)
     if (!aligned16(x)) return MALA_ERR_UNSUPPORTED;
-  const size_t need = mala_bwd_workspace_size(B, Hq, L, d);
+  const bool packed = pk.cu_q != nullptr;
+  const int tb = packed ? 1 : B, tl = packed ? pk.total_q : L;  // tensor extents [tb, tl, H, d]
+  const size_t need = mala_bwd_workspace_size(tb, Hq, tl, d);
   if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if (!make_bshd_map(&mq, q, B, L, Hq, d, 128) || !make_bshd_map(&mk, k, B, L, Hkv, d, 128) ||
-      !make_bshd_map(&mv, v, B, L, Hkv, d, 128) || !make_bshd_map(&mdo, dO, B, L, Hq, d, 128) ||
-      !make_bshd_map(&mdk, dk, B, L, Hkv, d, 128) || !make_bshd_map(&mdv, dv, B, L, Hkv, d, 128))
+  if (!make_bshd_map(&mq, q, tb, tl, Hq, d, 128) || !make_bshd_map(&mk, k, tb, tl, Hkv, d, 128) ||
+      !make_bshd_map(&mv, v, tb, tl, Hkv, d, 128) || !make_bshd_map(&mdo, dO, tb, tl, Hq, d, 128) ||
+      !make_bshd_map(&mdk, dk, tb, tl, Hkv, d, 128) || !make_bshd_map(&mdv, dv, tb, tl, Hkv, d, 128))
     return MALA_ERR_CUDA;
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
   float* dq_acc = static_cast<float*>(workspace);
   CUtensorMap mdq;
-  if (!make_dq_acc_map(&mdq, dq_acc, B, L, Hq, d)) return MALA_ERR_CUDA;
+  if (!make_dq_acc_map(&mdq, dq_acc, tb, tl, Hq, d)) return MALA_ERR_CUDA;
   float* dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                         align256(static_cast<size_t>(B) * L * Hq * d * 4));
+                                         align256(static_cast<size_t>(tb) * tl * Hq * d * 4));
   mala::BwdParams p;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
   p.nq = (L + Bq - 1) / Bq;
@@ -340,31 +379,66 @@ int mala_bwd(const void* q, const void* k, const void* v, const void* o, const v
   p.lse = lse;
   p.dvec = dvec;
   p.dq_acc = dq_acc;
+  p.cu = pk.cu_q;
+  p.total = pk.total_q;
+  p.dk_out = static_cast<uint16_t*>(dk);
+  p.dv_out = static_cast<uint16_t*>(dv);
   p.kept_tiles = kept_tiles;
   p.keep_map = keep_map;
   p.status = status;
 
-  const long long chunks = static_cast<long long>(B) * L * Hq * (d / 8);  // 16-byte chunks of O / dO
+  const long long chunks = static_cast<long long>(tb) * tl * Hq * (d / 8);  // 16-byte chunks of O / dO
   const int pre_grid = static_cast<int>(std::min<long long>((chunks + 255) / 256, 148LL * 16));
   if (d == 128)
     mala::mala_bwd_pre_kernel<128><<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(o),
-        static_cast<const uint4*>(dO), dvec, reinterpret_cast<float4*>(dq_acc), kept_tiles, B, L, Hq);
+        static_cast<const uint4*>(dO), dvec, reinterpret_cast<float4*>(dq_acc), kept_tiles, B * Hq, tb, tl, Hq);
   else
     mala::mala_bwd_pre_kernel<64><<<pre_grid, 256, 0, st>>>(static_cast<const uint4*>(o),
-        static_cast<const uint4*>(dO), dvec, reinterpret_cast<float4*>(dq_acc), kept_tiles, B, L, Hq);
+        static_cast<const uint4*>(dO), dvec, reinterpret_cast<float4*>(dq_acc), kept_tiles, B * Hq, tb, tl, Hq);
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
 
   const bool gate = tau > 0.f;
+  int rc;
   if (d == 128) rc = launch_bwd_tiles<128>(Bq, Bk, gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
   else rc = launch_bwd_tiles<64>(Bq, Bk, gate, mq, mk, mv, mdo, mdk, mdv, mdq, p, st);
   if (rc != MALA_OK) return rc;
 
-  const long long n8 = static_cast<long long>(B) * L * Hq * d / 8;
+  const long long n8 = static_cast<long long>(tb) * tl * Hq * d / 8;
   const int cv_grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
   mala::mala_dq_convert_kernel<<<cv_grid, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
                                                          static_cast<uint4*>(dq), n8);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
+}  // namespace
+
+int mala_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int L, int d, float scale, float tau, int Bq,
+             int Bk, void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
+             void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  return run_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace,
+                 workspace_bytes, kept_tiles, keep_map, stream);
+}
+
+int mala_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                    void* dq, void* dk, void* dv, const int32_t* cu_seqlens, int num_seqs, int max_seqlen,
+                    int total, int Hq, int Hkv, int d, float scale, float tau, int Bq, int Bk, void* workspace,
+                    size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !kept_tiles || !cu_seqlens)
+    return MALA_ERR_INVALID_ARG;
+  if (num_seqs < 1 || max_seqlen < 1 || total < 1 || max_seqlen > total) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(1, Hq, Hkv, total, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  if (static_cast<long long>(num_seqs) * Hq >= (1ll << 24)) return MALA_ERR_UNSUPPORTED;
+  Packed pk;
+  pk.cu_q = pk.cu_k = cu_seqlens;
+  pk.total_q = pk.total_k = total;
+  return run_bwd(q, k, v, o, dO, lse, dq, dk, dv, num_seqs, Hq, Hkv, max_seqlen, d, scale, tau, Bq, Bk,
+                 workspace, workspace_bytes, kept_tiles, keep_map, stream, pk);
+}
+
 size_t mala_decode_workspace_size(int B, int Hq, int d, int n_splits) {
   if (B < 1 || Hq < 1 || n_splits < 1 || (d != 64 && d != 128)) return 0;
   const size_t parts = static_cast<size_t>(B) * Hq * n_splits;
@@ -400,26 +474,34 @@ int mala_decode_default_splits(int B, int Hkv, int Lk, int Bk) {
   return static_cast<int>(best);
 }
 
-int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,
-                int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, void* workspace,
-                size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
-  if (!q || !kcache || !vcache || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+namespace {
+// Paged KV cache for decode (null block_table: a contiguous cache).
+struct Paged {
+  const int* seqlens = nullptr;
+  const int* block_table = nullptr;
+  int max_pages = 0, num_pages = 0;
+};
+
+int check_decode_args(const void* q, const void* kc, const void* vc, const void* o, const float* lse, int B,
+                      int Hq, int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits,
+                      const int32_t* kept_tiles) {
+  if (!q || !kc || !vc || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Lk < 1 || Hq % Hkv != 0 || n_splits < 0) return MALA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale) || !(tau >= 0.f) || !std::isfinite(tau)) return MALA_ERR_INVALID_ARG;
   if ((d != 64 && d != 128) || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
   if (Hq / Hkv > mala::kDecMaxG) return MALA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Lk * Hkv * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q, kcache, vcache, o, lse};
+  const void* ptrs[] = {q, kc, vc, o, lse};
   for (const void* x : ptrs)
     if (!aligned16(x)) return MALA_ERR_UNSUPPORTED;
-  if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk);
-  if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
-  const size_t need = mala_decode_workspace_size(B, Hq, d, n_splits);
-  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  CUtensorMap mk, mv;
-  if (!make_bshd_map(&mk, kcache, B, Lk, Hkv, d, Bk) || !make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk))
-    return MALA_ERR_CUDA;
+  return MALA_OK;
+}
+
+// Split kernel + combine into caller-provided partials (parts_base: o partials,
+// then the LSE partials 256 bytes aligned). Lk is the longest sequence's length.
+int run_decode(const void* q, const CUtensorMap& mk, const CUtensorMap& mv, void* o, float* lse, int B, int Hq,
+               int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, void* parts_base,
+               int32_t* kept_tiles, uint8_t* keep_map, cudaStream_t st, const Paged& pg = Paged()) {
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
   const size_t parts = static_cast<size_t>(B) * Hq * n_splits;
@@ -430,9 +512,14 @@ int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, 
   p.tiles_per_split = (p.nk + n_splits - 1) / n_splits;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.thr = tau > 0.f ? std::log2(tau) - std::log2(static_cast<float>(Lk)) : 0.f;
+  p.log2_tau = tau > 0.f ? std::log2(tau) : 0.f;
+  p.seqlens = pg.seqlens;
+  p.block_table = pg.block_table;
+  p.max_pages = pg.max_pages;
+  p.num_pages = pg.num_pages;
   p.q = static_cast<const uint16_t*>(q);
-  p.o_part = static_cast<float*>(workspace);
-  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(parts * d * 4));
+  p.o_part = static_cast<float*>(parts_base);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(parts_base) + align256(parts * d * 4));
   p.kept_tiles = kept_tiles;
   p.keep_map = keep_map;
   p.status = status;
@@ -455,6 +542,54 @@ int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, 
                                                                         n_splits);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
+}  // namespace
+
+int mala_decode(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,
+                int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, void* workspace,
+                size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  int rc = check_decode_args(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, kept_tiles);
+  if (rc != MALA_OK) return rc;
+  if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk);
+  if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
+  const size_t need = mala_decode_workspace_size(B, Hq, d, n_splits);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
+  CUtensorMap mk, mv;
+  if (!make_bshd_map(&mk, kcache, B, Lk, Hkv, d, Bk) || !make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk))
+    return MALA_ERR_CUDA;
+  return run_decode(q, mk, mv, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, workspace, kept_tiles,
+                    keep_map, static_cast<cudaStream_t>(stream));
+}
+
+int mala_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seqlens_k, void* o, float* lse, int B, int Hq, int Hkv, int num_pages,
+                      int page_size, int max_pages_per_seq, int d, float scale, float tau, int n_splits,
+                      void* workspace, size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map,
+                      void* stream) {
+  if (!block_table || !seqlens_k || num_pages < 1 || max_pages_per_seq < 1) return MALA_ERR_INVALID_ARG;
+  if (page_size != 64 && page_size != 128) return MALA_ERR_UNSUPPORTED;
+  const long long max_lk = static_cast<long long>(max_pages_per_seq) * page_size;
+  if (max_lk >= (1ll << 31) || static_cast<long long>(num_pages) * page_size >= (1ll << 31))
+    return MALA_ERR_UNSUPPORTED;
+  int rc = check_decode_args(q, k_pages, v_pages, o, lse, B, Hq, Hkv, static_cast<int>(max_lk), d, scale, tau,
+                             page_size, n_splits, kept_tiles);
+  if (rc != MALA_OK) return rc;
+  if (static_cast<long long>(num_pages) * page_size * Hkv * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
+  if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, static_cast<int>(max_lk), page_size);
+  if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
+  const size_t need = mala_decode_workspace_size(B, Hq, d, n_splits);
+  if (!workspace || workspace_bytes < need || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
+  CUtensorMap mk, mv;  // the pools as [num_pages, page, Hkv, d]: one page per tile
+  if (!make_bshd_map(&mk, k_pages, num_pages, page_size, Hkv, d, page_size) ||
+      !make_bshd_map(&mv, v_pages, num_pages, page_size, Hkv, d, page_size))
+    return MALA_ERR_CUDA;
+  Paged pg;
+  pg.seqlens = seqlens_k;
+  pg.block_table = block_table;
+  pg.max_pages = max_pages_per_seq;
+  pg.num_pages = num_pages;
+  return run_decode(q, mk, mv, o, lse, B, Hq, Hkv, static_cast<int>(max_lk), d, scale, tau, page_size, n_splits,
+                    workspace, kept_tiles, keep_map, static_cast<cudaStream_t>(stream), pg);
+}
 
 int mala_check_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -464,7 +599,8 @@ int mala_check_status(void* stream) {
   if (h != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_mala_status, &zero, sizeof(zero)) != cudaSuccess) return MALA_ERR_CUDA;
-    return (h & mala::kStatusTimeout) ? MALA_ERR_DEVICE_TIMEOUT : MALA_ERR_RANGE;
+    if (h & mala::kStatusTimeout) return MALA_ERR_DEVICE_TIMEOUT;
+    return (h & mala::kStatusSeqTable) ? MALA_ERR_INVALID_ARG : MALA_ERR_RANGE;
   }
   return MALA_OK;
 }
@@ -523,59 +659,19 @@ size_t mala_decode_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 int mala_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,
                         int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, int32_t* kept_tiles,
                         uint8_t* keep_map, void* stream) {
-  if (!q || !kcache || !vcache || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Lk < 1 || Hq % Hkv != 0 || n_splits < 0) return MALA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale) || !(tau >= 0.f) || !std::isfinite(tau)) return MALA_ERR_INVALID_ARG;
-  if ((d != 64 && d != 128) || (Bk != 64 && Bk != 128)) return MALA_ERR_UNSUPPORTED;
-  if (Hq / Hkv > mala::kDecMaxG) return MALA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * Lk * Hkv * d >= (1ll << 40)) return MALA_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q, kcache, vcache, o, lse};
-  for (const void* x : ptrs)
-    if (!aligned16(x)) return MALA_ERR_UNSUPPORTED;
+  int rc = check_decode_args(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, kept_tiles);
+  if (rc != MALA_OK) return rc;
   if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk);
   if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
   const size_t need = mala_decode_workspace_size(B, Hq, d, n_splits);
   if (need == 0 || need > kNoAllocScratchBytes) return MALA_ERR_WORKSPACE;  // beyond the fixed scratch
   void* scratch = decode_scratch_current_device();
   if (scratch == nullptr) return MALA_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap mk, mv;
   if (!make_bshd_map(&mk, kcache, B, Lk, Hkv, d, Bk) || !make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk))
     return MALA_ERR_CUDA;
-  unsigned* status = status_ptr();
-  if (!status) return MALA_ERR_CUDA;
-  const size_t parts = static_cast<size_t>(B) * Hq * n_splits;
-  mala::DecParams p;
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lk = Lk; p.G = Hq / Hkv;
-  p.nk = (Lk + Bk - 1) / Bk;
-  p.n_splits = n_splits;
-  p.tiles_per_split = (p.nk + n_splits - 1) / n_splits;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.thr = tau > 0.f ? std::log2(tau) - std::log2(static_cast<float>(Lk)) : 0.f;
-  p.q = static_cast<const uint16_t*>(q);
-  p.o_part = static_cast<float*>(scratch);
-  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + align256(parts * d * 4));
-  p.kept_tiles = kept_tiles;
-  p.keep_map = keep_map;
-  p.status = status;
-  if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
-  const bool gate = tau > 0.f;
-  int rc;
-  if (d == 128 && Bk == 128) rc = launch_dec_gate<128, 128>(gate, mk, mv, p, st);
-  else if (d == 64 && Bk == 128) rc = launch_dec_gate<64, 128>(gate, mk, mv, p, st);
-  else if (d == 128 && Bk == 64) rc = launch_dec_gate<128, 64>(gate, mk, mv, p, st);
-  else rc = launch_dec_gate<64, 64>(gate, mk, mv, p, st);
-  if (rc != MALA_OK) return rc;
-  const int rows = B * Hq;
-  if (d == 128)
-    mala::mala_decode_combine_kernel<128><<<(rows + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
-                                                                         static_cast<uint16_t*>(o), lse, rows,
-                                                                         n_splits);
-  else
-    mala::mala_decode_combine_kernel<64><<<(rows + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
-                                                                        static_cast<uint16_t*>(o), lse, rows,
-                                                                        n_splits);
-  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+  return run_decode(q, mk, mv, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, scratch, kept_tiles, keep_map,
+                    static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

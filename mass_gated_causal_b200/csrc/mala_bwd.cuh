@@ -45,8 +45,12 @@ struct BwdParams {
   int nq, nk, n_super;
   int chunk_kb;  // CTA schedule: key blocks per chunk (see mala_bwd_kernel)
   float scale, scale_log2, log2_tau;
-  const float* lse;   // [B, Hq, L]
-  const float* dvec;  // [B, Hq, L]: D_i
+  const float* lse;   // [B, Hq, L]; packed batches: [Hq, total]
+  const float* dvec;  // same layout as lse: D_i
+  const int* cu;      // packed batch (else null): sequence b owns rows cu[b] .. cu[b+1]; L is the longest
+  int total;          // packed batch: rows in all
+  uint16_t* dk_out;   // dK, dV (bf16), for the row-wise stores of a packed batch's partial key tiles
+  uint16_t* dv_out;
   float* dq_acc;      // [B, L, Hq, d] fp32 (the kernel adds into it through its tensor map)
   int32_t* kept_tiles;
   uint8_t* keep_map;
@@ -79,7 +83,9 @@ struct BwdLayout {
   static_assert(ALLOC_BYTES <= 232448, "backward shared memory exceeds the per-CTA limit");
 };
 
-template <int D, int BQ, int BK, bool kGate>
+// kPacked: a packed batch (p.cu set); the dense instantiation keeps every
+// length and offset a kernel parameter.
+template <int D, int BQ, int BK, bool kGate, bool kPacked>
 __global__ void __launch_bounds__(448, 1)
     mala_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -136,10 +142,25 @@ __global__ void __launch_bounds__(448, 1)
   const int in_chunk = static_cast<int>(blockIdx.x) % per_chunk;
   const int bk = in_chunk / p.chunk_kb;
   const int ks = chunk * p.chunk_kb + in_chunk % p.chunk_kb;
-  if (ks >= p.n_super) return;  // padding (uniform across the CTA, before any shared state)
   const int b = bk / p.Hkv, hkv = bk % p.Hkv;
+  // This CTA's sequence: L rows; a packed batch gives each sequence its own
+  // length and row offset (the grid covers the longest sequence, and a CTA past
+  // its sequence's rows leaves at once).
+  int L = p.L, off = 0, bt = b;
+  if (kPacked) {
+    off = __ldg(p.cu + b);
+    L = __ldg(p.cu + b + 1) - off;
+    bt = 0;
+    if (off < 0 || L < 0 || L > p.L || off + L > p.total) {  // nothing of this sequence is touched
+      if (threadIdx.x == 0 && ks == 0) atomicOr(p.status, kStatusSeqTable);
+      return;
+    }
+  }
+  const int n_super = (L + 127) / 128;
+  const int nq_b = (L + BQ - 1) / BQ, nk_b = (L + BK - 1) / BK;
+  if (ks >= n_super) return;  // padding (uniform across the CTA, before any shared state)
   const int k0 = ks * 128;
-  const int nqs = p.n_super - ks;
+  const int nqs = n_super - ks;
   const int T = p.G * nqs;
   // Walk order: the G query heads one after the other, each from the diagonal
   // query tile to the last. (Walking every CTA of a KV head through the same
@@ -187,8 +208,8 @@ __global__ void __launch_bounds__(448, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * TB);
       for (int h = 0; h < D / 64; ++h) {
-        tma_load_4d(&tm_k, kv_full, sK + h * 16384, h * 64, hkv, k0, b);
-        tma_load_4d(&tm_v, kv_full, sV + h * 16384, h * 64, hkv, k0, b);
+        tma_load_4d(&tm_k, kv_full, sK + h * 16384, h * 64, hkv, off + k0, bt);
+        tma_load_4d(&tm_v, kv_full, sV + h * 16384, h * 64, hkv, off + k0, bt);
       }
     }
     int issued_q = 0, issued_do = 0;
@@ -199,7 +220,7 @@ __global__ void __launch_bounds__(448, 1)
       const int i0 = walk_qs(t) * 128;
       if (lane == 0) {
         mbar_arrive_expect_tx(&q_full[st], TB);
-        for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_q, &q_full[st], sQ + st * TB + h * 16384, h * 64, hq, i0, b);
+        for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_q, &q_full[st], sQ + st * TB + h * 16384, h * 64, hq, off + i0, bt);
       }
       issued_q = t + 1;
       // dO of the same tile, before the gate has decided: the buffer is free as
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__(448, 1)
       if (t >= 1 && !mbar_wait_warp(do_empty, (t - 1) & 1, fs)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(do_full, TB);
-        for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, i0, b);
+        for (int h = 0; h < D / 64; ++h) tma_load_4d(&tm_do, do_full, sDO + h * 16384, h * 64, hq, off + i0, bt);
       }
       issued_do = t + 1;
     }
@@ -369,7 +390,8 @@ __global__ void __launch_bounds__(448, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (row0 < p.L) tma_reduce_add_4d(&tm_dq, buf, c * 32, hq, row0, b);  // rows past L are clipped
+            // rows past the tensor are clipped; rows past a packed sequence add exact zeros
+            if (row0 < L) tma_reduce_add_4d(&tm_dq, buf, c * 32, hq, off + row0, bt);
             bulk_commit();  // one group per block, empty when skipped, so the counting above holds
           }
         }
@@ -394,14 +416,18 @@ __global__ void __launch_bounds__(448, 1)
     const float sl2 = p.scale_log2;
     int nd = 0;
     bool local_abort = false, all_abort = false;
+    // LSE and D of query head hq start at row_base(hq): [B, Hq, L], or [Hq, total] for a packed batch
+    auto row_base = [&](int hq_) {
+      return kPacked ? static_cast<size_t>(hq_) * p.total + off : static_cast<size_t>(b * p.Hq + hq_) * L;
+    };
     // LSE and D of my row, loaded one tile ahead (rows at or past L: LSE +inf, D 0)
     auto row_lse = [&](int t) {
       const int i = walk_qs(t) * 128 + row;
-      return i < p.L ? __ldg(p.lse + static_cast<size_t>(b * p.Hq + walk_hq(t)) * p.L + i) : INFINITY;
+      return i < L ? __ldg(p.lse + row_base(walk_hq(t)) + i) : INFINITY;
     };
     auto row_d = [&](int t) {
       const int i = walk_qs(t) * 128 + row;
-      return i < p.L ? __ldg(p.dvec + static_cast<size_t>(b * p.Hq + walk_hq(t)) * p.L + i) : 0.f;
+      return i < L ? __ldg(p.dvec + row_base(walk_hq(t)) + i) : 0.f;
     };
     float lse_next = row_lse(0), d_next = row_d(0);
 
@@ -442,7 +468,7 @@ __global__ void __launch_bounds__(448, 1)
         hit = ok && m * sl2 >= thr;
       } else {
         const int qb = qs * QPB + qi, kb = ks * KPB + kx;
-        hit = qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1;
+        hit = qb < nq_b && kb < nk_b && kb * BK <= min((qb + 1) * BQ, L) - 1;
       }
       const unsigned bal = __ballot_sync(0xffffffffu, hit);
       if (lane == 0) vote[(t & 1) * 8 + warp] = (bal ? 1u : 0u) | (local_abort ? 8u : 0u);
@@ -468,7 +494,7 @@ __global__ void __launch_bounds__(448, 1)
         for (int qx = 0; qx < QPB; ++qx)
           for (int kz = 0; kz < KPB; ++kz) {
             const int qb = qs * QPB + qx, kb = ks * KPB + kz;
-            if (qb < p.nq && kb < p.nk && kb * BK <= min((qb + 1) * BQ, p.L) - 1) {
+            if (qb < nq_b && kb < nk_b && kb * BK <= min((qb + 1) * BQ, L) - 1) {
               const int kp = (kept >> (qx * 2 + kz)) & 1u;
               if (p.keep_map) p.keep_map[(static_cast<size_t>(b * p.Hq + hq) * p.nq + qb) * p.nk + kb] = kp;
               cnt += kp;
@@ -559,12 +585,29 @@ __global__ void __launch_bounds__(448, 1)
       uint32_t all_ok = 1u;
 #pragma unroll
       for (int w = 0; w < 8; ++w) all_ok &= evote[w];
-      if (tid == 0 && all_ok) {
+      // A packed batch's partial key tile is stored row by row: a tile store
+      // would write the next sequence's rows.
+      const bool whole = !kPacked || k0 + 128 <= L;
+      if (whole && tid == 0 && all_ok) {
         for (int h = 0; h < D / 64; ++h) {
-          tma_store_4d(&tm_dk, sQ + h * 16384, h * 64, hkv, k0, b);
-          tma_store_4d(&tm_dv, sQ + TB + h * 16384, h * 64, hkv, k0, b);
+          tma_store_4d(&tm_dk, sQ + h * 16384, h * 64, hkv, off + k0, bt);
+          tma_store_4d(&tm_dv, sQ + TB + h * 16384, h * 64, hkv, off + k0, bt);
         }
         tma_store_commit_and_wait();
+      }
+      if (!whole && all_ok && k0 + row < L) {
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          uint4* dst = reinterpret_cast<uint4*>((which == 0 ? p.dk_out : p.dv_out) +
+                                                (static_cast<size_t>(off + k0 + row) * p.Hkv + hkv) * D);
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            const int col = kh * (D / 2) + c * 8;
+            uint32_t a0, a1, a2, a3;
+            ld_shared_v4(sQa + which * TB + (col >> 6) * 16384 + sw128_offset(row, (col & 63) >> 3), a0, a1, a2, a3);
+            dst[col / 8] = make_uint4(a0, a1, a2, a3);
+          }
+        }
       }
     }
   }
@@ -584,7 +627,8 @@ __global__ void __launch_bounds__(448, 1)
 template <int D>
 __global__ void __launch_bounds__(256) mala_bwd_pre_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dO,
                                                           float* __restrict__ dvec, float4* __restrict__ dq_acc,
-                                                          int32_t* __restrict__ kept, int B, int L, int Hq) {
+                                                          int32_t* __restrict__ kept, int n_kept, int B, int L,
+                                                          int Hq) {
   constexpr int TPR = D / 8;
   const long long total = static_cast<long long>(B) * L * Hq * TPR;
   const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -622,7 +666,7 @@ __global__ void __launch_bounds__(256) mala_bwd_pre_kernel(const uint4* __restri
     }
   }
   if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < B * Hq; i += blockDim.x) kept[i] = 0;
+    for (int i = threadIdx.x; i < n_kept; i += blockDim.x) kept[i] = 0;
 }
 
 // bf16 dQ from the fp32 accumulator (the softmax scale is already applied).

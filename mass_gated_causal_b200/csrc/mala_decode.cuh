@@ -37,9 +37,15 @@ constexpr int kDecMaxG = 8;  // query heads per KV head handled by one CTA
 constexpr int kDecLag = 2;   // kept tiles between a tile's gate and its PV
 
 struct DecParams {
-  int B, Hq, Hkv, Lk, G, nk, n_splits, tiles_per_split;
+  int B, Hq, Hkv, Lk, G, nk, n_splits, tiles_per_split;  // paged cache: Lk, nk = the longest sequence's
   float scale_log2;
-  float thr;  // log2(tau) - log2(Lk)
+  float thr;       // log2(tau) - log2(Lk)
+  float log2_tau;  // paged cache: the threshold is formed per sequence
+  // paged cache (else null): sequence b's key tile kb is page block_table[b * max_pages + kb] of the
+  // [num_pages, page = Bk, Hkv, d] pools, its length seqlens[b]
+  const int* seqlens;
+  const int* block_table;
+  int max_pages, num_pages;
   const uint16_t* q;  // [B, Hq, d] bf16
   float* o_part;      // [B, Hq, S, d]
   float* lse_part;    // [B, Hq, S] natural log
@@ -105,7 +111,9 @@ struct DecLayout {
   static_assert(ALLOC_BYTES <= 232448, "decode shared memory exceeds the per-CTA limit");
 };
 
-template <int D, int BK, int GP, bool kGate>
+// kPaged: a paged cache (p.seqlens and p.block_table set); the contiguous
+// instantiation keeps every length a kernel parameter.
+template <int D, int BK, int GP, bool kGate, bool kPaged>
 __global__ void __launch_bounds__(320, 1)
     mala_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                              const DecParams p) {
@@ -144,10 +152,37 @@ __global__ void __launch_bounds__(320, 1)
   const int b = bk / p.Hkv, hkv = bk % p.Hkv;
   const int G = p.G;
   const int hq0 = hkv * G;
-  const int t0 = min(sp_idx * p.tiles_per_split, p.nk);
-  const int t1 = min(t0 + p.tiles_per_split, p.nk);
+  // this sequence's keys: Lk of them in nk tiles (a paged cache gives each its own)
+  int Lk = p.Lk, nk = p.nk, tps = p.tiles_per_split;
+  bool bad = false;
+  if (kPaged) {
+    Lk = __ldg(p.seqlens + b);
+    bad = Lk < 1 || Lk > p.Lk;
+    if (bad) Lk = 1;
+    nk = (Lk + BK - 1) / BK;
+    tps = (nk + p.n_splits - 1) / p.n_splits;
+  }
+  const float thr = kPaged ? p.log2_tau - log2f(static_cast<float>(Lk)) : p.thr;  // log2(tau / Lq), Lq = Lk
+  const int t0 = bad ? nk : min(sp_idx * tps, nk);
+  const int t1 = bad ? nk : min(t0 + tps, nk);
   const int T = t1 - t0;  // tiles kb = t1-1 ... t0
   const FailState fs{abort_flag, p.status};
+  // TMA coordinates (row, outer index) of key tile kb: a page of the pool, or rows of sequence b
+  auto tile_at = [&](int kb, int& row, int& outer) {
+    if (kPaged) {
+      const int pg = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + kb);
+      row = 0;
+      outer = pg;
+      if (pg < 0 || pg >= p.num_pages) {  // read as zeros (a load outside the tensor fills), reported
+        atomicOr(p.status, kStatusSeqTable);
+        outer = p.num_pages;
+      }
+    } else {
+      row = kb * BK;
+      outer = b;
+    }
+  };
+  if (bad && sp_idx == 0 && tid == 0) atomicOr(p.status, kStatusSeqTable);
 
   if (T <= 0) {  // empty split: contributes nothing to the merge
     for (int i = tid; i < G * D; i += blockDim.x) {
@@ -185,9 +220,11 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < T; ++t) {
         const int st = t % NK;
         if (t >= NK && !mbar_wait(&k_empty[st], ((t / NK) - 1) & 1, fs)) break;
+        int krow, kouter;
+        tile_at(t1 - 1 - t, krow, kouter);
         mbar_arrive_expect_tx(&k_full[st], TB);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(&tm_k, &k_full[st], sK + st * TB + h * (BK * 128), h * 64, hkv, (t1 - 1 - t) * BK, b);
+          tma_load_4d(&tm_k, &k_full[st], sK + st * TB + h * (BK * 128), h * 64, hkv, krow, kouter);
         issued = t + 1;
       }
       for (int t = max(0, issued - NK); t < issued; ++t) mbar_wait_drain(&k_full[t % NK], (t / NK) & 1);
@@ -214,7 +251,7 @@ __global__ void __launch_bounds__(320, 1)
           sum += sRsum[w * GP + g];
         }
         float l = sL[g] + sum, mu = sM[g];
-        keep = (t == 0) || !kGate || (M * p.scale_log2 >= mu + lg2_approx(l) + p.thr);
+        keep = (t == 0) || !kGate || (M * p.scale_log2 >= mu + lg2_approx(l) + thr);
         float alpha = 1.f;
         if (keep) {
           const float mnew = fmaxf(mu, M * p.scale_log2);
@@ -238,10 +275,12 @@ __global__ void __launch_bounds__(320, 1)
         const bool ab = abort_raised(fs);
         if (any && !ab) {  // V is requested only now that a head keeps the tile
           const int vs = nkept % NV;
+          int vrow, vouter;
+          tile_at(kb, vrow, vouter);
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(&v_full[vs], TB);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(&tm_v, &v_full[vs], sV + vs * TB + h * (BK * 128), h * 64, hkv, kb * BK, b);
+            tma_load_4d(&tm_v, &v_full[vs], sV + vs * TB + h * (BK * 128), h * 64, hkv, vrow, vouter);
         }
         *sflag = (any ? 1u : 0u) | (ab ? 2u : 0u);
         aborted = ab;
@@ -330,7 +369,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       const float mine = group_reduce_scatter<GP, LPK>(part, c);  // score of key j for my head hh
-      const bool live = kb * BK + j < p.Lk;
+      const bool live = kb * BK + j < Lk;
       if (live) mx = fmaxf(mx, mine);
       sc[s2] = live ? mine : -INFINITY;
     }

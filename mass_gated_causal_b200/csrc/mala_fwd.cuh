@@ -52,7 +52,11 @@ struct FwdParams {
   int chunk_pairs;      // CTA schedule: pairs per chunk (see mala_fwd_kernel)
   float scale_log2;     // scale * log2(e): scores are kept in log2 units
   float log2_tau;       // log2(tau), used only when the gate is on
-  float* lse;           // [B, Hq, L]
+  float* lse;           // [B, Hq, Lq]; packed batches: [Hq, total_q]
+  uint16_t* o;          // the output (bf16), for the row-wise stores of a packed batch's partial tiles
+  const int* cu_q;      // packed batch (else null): sequence b owns query rows cu_q[b] .. cu_q[b+1]
+  const int* cu_k;      //   and key rows cu_k[b] .. cu_k[b+1] of the packed tensors
+  int total_q, total_k; // packed batch: query and key rows in all
   int32_t* kept_tiles;
   uint8_t* keep_map;
   unsigned* status;
@@ -144,13 +148,31 @@ __global__ void __launch_bounds__(320, 1)
   const int chunk = static_cast<int>(blockIdx.x) / per_chunk;
   const int in_chunk = static_cast<int>(blockIdx.x) % per_chunk;
   const int unit = in_chunk / per_unit;
-  const int pr = p.n_pairs - 1 - (chunk * p.chunk_pairs + (in_chunk % per_unit) / p.G);
-  if (pr < 0) return;  // padding (uniform across the CTA, before any shared state)
   const int b = unit / p.Hkv, hkv = unit % p.Hkv, hq = hkv * p.G + in_chunk % p.G;
   const int bh = b * p.Hq + hq;
+  // This CTA's sequence: Lq queries at positions P0 .. P0 + Lq - 1 of Lk keys.
+  // A packed batch gives each sequence its own lengths and row offsets into the
+  // packed tensors (its pairs are counted from its own last row; the grid covers
+  // the longest sequence, and a CTA past its sequence's rows leaves at once).
+  int Lq = p.Lq, Lk = p.Lk, q_off = 0, k_off = 0, bt = b;
+  if (p.cu_q != nullptr) {  // p.Lq / p.Lk hold the longest sequence's lengths
+    q_off = __ldg(p.cu_q + b);
+    Lq = __ldg(p.cu_q + b + 1) - q_off;
+    k_off = __ldg(p.cu_k + b);
+    Lk = __ldg(p.cu_k + b + 1) - k_off;
+    bt = 0;
+    if (q_off < 0 || Lq < 0 || Lq > p.Lq || q_off + Lq > p.total_q || k_off < 0 || Lk < Lq || Lk > p.Lk ||
+        k_off + Lk > p.total_k) {  // nothing of this sequence is touched
+      if (threadIdx.x == 0) atomicOr(p.status, kStatusSeqTable);
+      return;
+    }
+  }
+  const int P0 = Lk - Lq;
+  const int pr = (Lq + 2 * BM - 1) / (2 * BM) - 1 - (chunk * p.chunk_pairs + (in_chunk % per_unit) / p.G);
+  if (pr < 0) return;  // padding (uniform across the CTA, before any shared state)
   const int r0 = pr * 2 * BM;  // first row of tile A
-  const int last_row = min(r0 + 2 * BM, p.Lq) - 1;  // among the queries
-  const int kb_hi = (p.P0 + last_row) / BK;         // key tile of the pair's last query
+  const int last_row = min(r0 + 2 * BM, Lq) - 1;  // among the queries
+  const int kb_hi = (P0 + last_row) / BK;         // key tile of the pair's last query
   const int T = kb_hi + 1;
 
   if (threadIdx.x == 0) {
@@ -189,7 +211,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive_expect_tx(bar_q, 2 * Lay::Q_BYTES);
       for (int x = 0; x < 2; ++x)
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(&tm_q, bar_q, sQ + x * Lay::Q_BYTES + h * (BM * 128), h * 64, hq, r0 + x * BM, b);
+          tma_load_4d(&tm_q, bar_q, sQ + x * Lay::Q_BYTES + h * (BM * 128), h * 64, hq, q_off + r0 + x * BM, bt);
       int issued = 0, vissued = 0;
       for (int t = 0; t < T; ++t) {
         const int st = t % NK;
@@ -197,7 +219,8 @@ __global__ void __launch_bounds__(320, 1)
         if (t >= NK && !mbar_wait(&k_empty[st], ((t / NK) - 1) & 1, fs)) break;
         mbar_arrive_expect_tx(&k_full[st], Lay::KV_BYTES);
         for (int h = 0; h < D / 64; ++h)
-          tma_load_4d(&tm_k, &k_full[st], sK + st * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, kb * BK, b);
+          tma_load_4d(&tm_k, &k_full[st], sK + st * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, k_off + kb * BK,
+                      bt);
         issued = t + 1;
         // V(t) is fetched ahead into slot t % NV whatever the vote decides
         // (see the note on V above)
@@ -206,7 +229,8 @@ __global__ void __launch_bounds__(320, 1)
           if (t >= NV && !mbar_wait(&v_empty[vs], ((t / NV) - 1) & 1, fs)) break;
           mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(&tm_v, &v_full[vs], sV + vs * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, kb * BK, b);
+            tma_load_4d(&tm_v, &v_full[vs], sV + vs * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, k_off + kb * BK,
+                      bt);
           vissued = t + 1;
         }
       }
@@ -283,12 +307,12 @@ __global__ void __launch_bounds__(320, 1)
     const int wq = warp & 3;            // TMEM lane quarter
     const int row0 = r0 + x * BM;
     const int row = row0 + tid;
-    const bool row_ok = row < p.Lq;
-    const int pos = p.P0 + row;  // the query's position: it sees keys 0 .. pos
+    const bool row_ok = row < Lq;
+    const int pos = P0 + row;  // the query's position: it sees keys 0 .. pos
     const int qi = tid / BQ;
     const int qb = (row0 / BQ) + qi;
-    const bool blk_exists = qb < p.nq;
-    const int kbf = blk_exists ? (p.P0 + min((qb + 1) * BQ, p.Lq) - 1) / BK : -1;
+    const bool blk_exists = qb < (Lq + BQ - 1) / BQ;
+    const int kbf = blk_exists ? (P0 + min((qb + 1) * BQ, Lq) - 1) / BK : -1;
     const float thr = kGate ? p.log2_tau - lg2_approx(static_cast<float>(pos + 1)) : 0.f;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + Lay::COL_S + x * BK + lane_base;
@@ -305,7 +329,7 @@ __global__ void __launch_bounds__(320, 1)
       const bool ok = mbar_wait_warp(&s_full[x], t & 1, fs);
       local_abort |= !ok;
       tc_fence_after();
-      const bool diag = kb * BK + BK - 1 > p.P0 + row0;  // some key of the tile is past some row
+      const bool diag = kb * BK + BK - 1 > P0 + row0;  // some key of the tile is past some row
       // first pass (row max): all loads of the S row in flight at once, one wait
       float M = -INFINITY;
       {
@@ -459,16 +483,30 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         fence_proxy_async_smem();
-        if (row_ok) p.lse[static_cast<size_t>(bh) * p.Lq + row] = (m_use + lg2_approx(l)) * 0.69314718055994531f;
+        const size_t lse_at = p.cu_q != nullptr ? static_cast<size_t>(hq) * p.total_q + q_off + row
+                                                : static_cast<size_t>(bh) * Lq + row;
+        if (row_ok) p.lse[lse_at] = (m_use + lg2_approx(l)) * 0.69314718055994531f;
       }
       const unsigned okall = __ballot_sync(0xffffffffu, okf);
       if (lane == 0) evote[x * 4 + wq] = okall == 0xffffffffu ? 1u : 0u;
       named_bar_sync(1 + x, 128);
       const bool store = (evote[x * 4 + 0] & evote[x * 4 + 1] & evote[x * 4 + 2] & evote[x * 4 + 3]) != 0;
-      if (tid == 0 && store && row0 < p.Lq) {
+      // A packed batch's partial tile is stored row by row: a tile store would
+      // write the next sequence's rows.
+      const bool whole = p.cu_q == nullptr || row0 + BM <= Lq;
+      if (whole && tid == 0 && store && row0 < Lq) {
         for (int h = 0; h < D / 64; ++h)
-          tma_store_4d(&tm_o, sQ + x * Lay::Q_BYTES + h * (BM * 128), h * 64, hq, row0, b);
+          tma_store_4d(&tm_o, sQ + x * Lay::Q_BYTES + h * (BM * 128), h * 64, hq, q_off + row0, bt);
         tma_store_commit_and_wait();
+      }
+      if (!whole && store && row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(q_off + row) * p.Hq + hq) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          uint32_t a0, a1, a2, a3;
+          ld_shared_v4(sQa + (c >> 3) * (BM * 128) + sw128_offset(tid, c & 7), a0, a1, a2, a3);
+          dst[c] = make_uint4(a0, a1, a2, a3);
+        }
       }
       if ((tid % BQ) == 0 && blk_exists && store) atomicAdd(&p.kept_tiles[bh], kept_count);
     }

@@ -18,6 +18,7 @@ namespace mala {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusSeqTable = 4u;  // a packed batch's sequence table or page table was invalid
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

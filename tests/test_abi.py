@@ -76,6 +76,64 @@ def test_prefill_rejects(kw, code):
     assert pre(**kw) == code
 
 
+def fvl(**kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, cu_seqlens_q=P, cu_seqlens_k=P, num_seqs=3, max_seqlen_q=100,
+             max_seqlen_k=200, total_q=250, total_k=400, Hq=4, Hkv=2, d=128, scale=0.1, tau=1.0, Bq=128, Bk=64,
+             workspace=P, workspace_bytes=1 << 30, kept_tiles=P, keep_map=None, stream=S)
+    a.update(kw)
+    return mala.mala_fwd_varlen(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu_seqlens_q=None), 1), (dict(cu_seqlens_k=None), 1), (dict(lse=None), 1), (dict(num_seqs=0), 1),
+    (dict(max_seqlen_q=0), 1), (dict(total_k=0), 1), (dict(max_seqlen_q=300), 1), (dict(max_seqlen_k=500), 1),
+    (dict(Hq=3), 1), (dict(tau=-1.0), 1),
+    (dict(d=32), 2), (dict(Bq=32), 2), (dict(v=P + 8), 2),
+    (dict(workspace=None), 3), (dict(workspace=P + 64), 3),
+    # the fp16 V copy covers all total_k key rows
+    (dict(workspace_bytes=(400 * 2 * 128 * 2 + 255) // 256 * 256 - 1), 3),
+])
+def test_fwd_varlen_rejects(kw, code):
+    assert fvl(**kw) == code
+
+
+def bvl(**kw):
+    a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, cu_seqlens=P, num_seqs=2, max_seqlen=300, total=400,
+             Hq=4, Hkv=2, d=64, scale=0.1, tau=1.0, Bq=64, Bk=128, workspace=P, workspace_bytes=1 << 30,
+             kept_tiles=P, keep_map=None, stream=S)
+    a.update(kw)
+    return mala.mala_bwd_varlen(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu_seqlens=None), 1), (dict(dk=None), 1), (dict(num_seqs=0), 1), (dict(max_seqlen=401), 1),
+    (dict(total=0), 1), (dict(Hq=5), 1), (dict(d=100), 2), (dict(Bk=96), 2), (dict(dq=P + 2), 2),
+    (dict(workspace=None), 3),
+    (dict(workspace_bytes=(400 * 4 * 64 * 4 + 255) // 256 * 256 + (4 * 400 * 4 + 255) // 256 * 256 - 1), 3),
+])
+def test_bwd_varlen_rejects(kw, code):
+    assert bvl(**kw) == code
+
+
+def dpg(**kw):
+    a = dict(q=P, k_pages=P, v_pages=P, block_table=P, seqlens_k=P, o=P, lse=P, B=4, Hq=8, Hkv=2, num_pages=100,
+             page_size=128, max_pages_per_seq=40, d=128, scale=0.1, tau=1.0, n_splits=4, workspace=P,
+             workspace_bytes=1 << 30, kept_tiles=P, keep_map=None, stream=S)
+    a.update(kw)
+    return mala.mala_decode_paged(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(block_table=None), 1), (dict(seqlens_k=None), 1), (dict(num_pages=0), 1), (dict(max_pages_per_seq=0), 1),
+    (dict(q=None), 1), (dict(Hq=6, Hkv=4), 1), (dict(n_splits=-2), 1),
+    (dict(page_size=32), 2), (dict(page_size=256), 2), (dict(d=96), 2), (dict(Hq=64, Hkv=2), 2),
+    (dict(max_pages_per_seq=1 << 24), 2), (dict(k_pages=P + 8), 2),
+    (dict(workspace=None), 3), (dict(workspace_bytes=64), 3),
+])
+def test_decode_paged_rejects(kw, code):
+    assert dpg(**kw) == code
+
+
 def bwd(**kw):
     a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, B=1, Hq=2, Hkv=1, L=100, d=128, scale=0.1,
              tau=1.0, Bq=128, Bk=128, workspace=P, workspace_bytes=1 << 30, kept_tiles=P, keep_map=None, stream=S)
