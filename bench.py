@@ -38,7 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import C2, C3, C4, WORKLOADS, default_workers  # noqa: E402
+from workloads import C2, C3, C4, C5, WORKLOADS, default_workers  # noqa: E402
 
 METRIC = "MALA fwd+bwd ms & eff. TFLOP/s (% bf16 peak) at 32K/128K, τ=1; retained-tile %"
 L2_BYTES = 126 * 1024 * 1024
@@ -331,6 +331,11 @@ def run_cuda(args):
     if not args.no_long and w.name != C3.name:
         long_leg = run_train_leg(C3, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world)
 
+    # a packed batch of mixed lengths (32K tokens in all)
+    varlen_leg = None
+    if not args.no_varlen:
+        varlen_leg = run_varlen_leg(C5, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world)
+
     # decode workload
     dec = None
     if not args.no_decode:
@@ -386,6 +391,8 @@ def run_cuda(args):
     }
     if long_leg is not None:
         line["at_128k"] = long_leg
+    if varlen_leg is not None:
+        line["varlen"] = varlen_leg
     if dec is not None:
         line["decode"] = dec
     if cpu is not None:
@@ -459,6 +466,127 @@ def run_train_leg(w, mala, torch, dev, stream, pk, workers, timed, max_over_rank
     return out
 
 
+def run_varlen_leg(w, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world, steps=3, warmup=3):
+    """fwd+bwd of a packed batch (mala_fwd_varlen + mala_bwd_varlen) at tau = 1 and tau = 0."""
+    from workloads import make_packed_inputs
+    inp = make_packed_inputs(w, workers=workers)
+    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v, do = (to_dev(inp[x]) for x in ("q", "k", "v", "do"))
+    cu = torch.from_numpy(inp["cu_seqlens"]).to(dev)
+    del inp
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    S, Lmax = len(w.lens), max(w.lens)
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    kept_f = torch.empty((S * Hq,), dtype=torch.int32, device=dev)
+    kept_b = torch.empty((S * Hq,), dtype=torch.int32, device=dev)
+    ws_bytes = mala.mala_bwd_workspace_size(1, Hq, T, d)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    fws_bytes = mala.mala_fwd_workspace_size(1, Hkv, T, d)
+    fws = torch.empty((fws_bytes,), dtype=torch.uint8, device=dev)
+    nq, nk = -(-Lmax // w.Bq), -(-Lmax // w.Bk)
+
+    def step(tau_, km_f=None, km_b=None, mid=None):
+        rc = mala.mala_fwd_varlen(q, k, v, o, lse, cu, cu, S, Lmax, Lmax, T, T, Hq, Hkv, d, w.scale, tau_, w.Bq, w.Bk,
+                                  fws, fws_bytes, kept_f, km_f, stream)
+        assert rc == 0, mala.mala_status_string(rc)
+        if mid is not None:
+            mid.record(stream)
+        rc = mala.mala_bwd_varlen(q, k, v, o, do, lse, dq, dk, dv, cu, S, Lmax, T, Hq, Hkv, d, w.scale, tau_, w.Bq,
+                                  w.Bk, ws, ws_bytes, kept_b, km_b, stream)
+        assert rc == 0, mala.mala_status_string(rc)
+
+    km_f = torch.zeros((S, Hq, nq, nk), dtype=torch.uint8, device=dev)
+    km_b = torch.zeros((S, Hq, nq, nk), dtype=torch.uint8, device=dev)
+    step(1.0, km_f, km_b)
+    assert mala.mala_check_status(stream) == 0
+    kmf, kmb = km_f.cpu().numpy(), km_b.cpu().numpy()
+    del km_f, km_b
+    fl = {"n_legal": 0, "n_f": 0, "n_b": 0, "fwd": 0, "bwd": 0}
+    fl0 = dict(fl)
+    n_tiles = kept_tf = kept_tb = 0
+    for s_, L in enumerate(w.lens):  # per sequence: its own live pairs and its corner of the keep maps
+        live = live_pairs(L, w.Bq, w.Bk)
+        a, b_ = live.shape
+        f1 = train_flops(d, 1, Hq, L, live, kmf[s_:s_ + 1, :, :a, :b_], kmb[s_:s_ + 1, :, :a, :b_])
+        f0 = train_flops(d, 1, Hq, L, live, None, None)
+        for key_ in fl:
+            fl[key_] += f1[key_]
+            fl0[key_] += f0[key_]
+        n_tiles += Hq * int((live > 0).sum())
+        kept_tf += int((kmf[s_, :, :a, :b_] == 1).sum())
+        kept_tb += int((kmb[s_, :, :a, :b_] == 1).sum())
+    out = {"workload": w.name, "lens": list(w.lens), "total": T, "Hq": Hq, "Hkv": Hkv, "d": d, "Bq": w.Bq,
+           "Bk": w.Bk, "steps": steps, "warmup": warmup,
+           "retained_tiles": {"fwd": round(kept_tf / n_tiles, 4), "bwd": round(kept_tb / n_tiles, 4),
+                              "live_pair_frac_fwd": round(fl["n_f"] / fl["n_legal"], 4),
+                              "live_pair_frac_bwd": round(fl["n_b"] / fl["n_legal"], 4)}}
+    peak_t = pk["bf16_tflops_sustained"]
+    for tau_, flops, key in ((1.0, fl["fwd"] + fl["bwd"], "tau1"), (0.0, fl0["fwd"] + fl0["bwd"], "tau0")):
+        tot, f, b_ = timed(lambda mid=None, t_=tau_: step(t_, mid=mid), steps, warmup)
+        ms = max_over_ranks(float(np.mean(tot)))
+        tf = world * flops / (ms * 1e-3) / 1e12
+        out[key] = {"ms_per_step": round(ms, 3), "fwd_ms": round(max_over_ranks(float(np.mean(f))), 3),
+                    "bwd_ms": round(max_over_ranks(float(np.mean(b_))), 3), "tflops": round(tf, 2),
+                    "frac_of_peak": round(tf / world / peak_t, 4)}
+    assert mala.mala_check_status(stream) == 0
+    out["mala_speedup"] = round(out["tau0"]["ms_per_step"] / out["tau1"]["ms_per_step"], 3)
+    return out
+
+
+def run_paged_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, contiguous):
+    """The decode workload's cache scattered into shuffled page pools (page = Bk):
+    the same bytes as the contiguous decode, read through the block table."""
+    B, Hq, d = q.shape
+    Lk, Hkv = kc.shape[1], kc.shape[2]
+    page = w.Bk
+    npg = -(-Lk // page)
+    assert npg * page == Lk
+    g = torch.Generator().manual_seed(w.seed + 77)
+    perm = torch.randperm(B * npg, generator=g).to(dev)
+    kp = torch.empty((B * npg, page, Hkv, d), dtype=kc.dtype, device=dev)
+    vp = torch.empty_like(kp)
+    kp[perm] = kc.reshape(B * npg, page, Hkv, d)
+    vp[perm] = vc.reshape(B * npg, page, Hkv, d)
+    table = perm.to(torch.int32).reshape(B, npg).contiguous()
+    sl = torch.full((B,), Lk, dtype=torch.int32, device=dev)
+    ns = contiguous["n_splits"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    kept = torch.empty((B * Hq,), dtype=torch.int32, device=dev)
+    wsb = mala.mala_decode_workspace_size(B, Hq, d, ns)
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+    out = {"workload": w.name + "_paged", "page": page, "num_pages": B * npg, "n_splits": ns,
+           "layout": "pages shuffled over the pool (seeded permutation)"}
+    for tau in (1.0, 0.0):
+        km = torch.zeros((B, Hq, npg), dtype=torch.uint8, device=dev)
+        rc = mala.mala_decode_paged(q, kp, vp, table, sl, o, lse, B, Hq, Hkv, B * npg, page, npg, d, w.scale, tau, ns,
+                                    ws, wsb, kept, km, stream)
+        assert rc == 0
+        assert mala.mala_check_status(stream) == 0
+        by = decode_bytes(B, Hq, Hkv, Lk, d, page, km.cpu().numpy())
+        del km
+
+        def fn(mid=None, tau_=tau):
+            rc_ = mala.mala_decode_paged(q, kp, vp, table, sl, o, lse, B, Hq, Hkv, B * npg, page, npg, d, w.scale, tau_,
+                                         ns, ws, wsb, kept, None, stream)
+            assert rc_ == 0
+            if mid is not None:
+                mid.record(stream)
+        tot, _, _ = timed(fn, max(5, args.steps * 2), max(3, args.warmup))
+        us = max_over_ranks(float(np.median(tot))) * 1e3
+        gbs = by["total"] / (us * 1e-6) / 1e9
+        key = f"tau{int(tau)}"
+        out[key] = {"us_per_step": round(us, 1), "us_per_token": round(us / B, 2), "GBps": round(gbs, 1),
+                    "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "bytes_per_step": by["total"],
+                    "vs_contiguous": round(contiguous[key]["us_per_step"] / us, 3)}
+    assert mala.mala_check_status(stream) == 0
+    del kp, vp
+    return out
+
+
 def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world):
     from workloads import make_decode_inputs
     w = C4
@@ -502,6 +630,7 @@ def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_rank
                                  "retained_tile_frac_per_head": round(float((kmh == 1).mean()), 4)}
     out["mala_speedup"] = round(out["tau0"]["us_per_step"] / out["tau1"]["us_per_step"], 3)
     out["hbm_peak_gbs"] = pk["hbm_gbs"]
+    out["paged"] = run_paged_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, out)
     return out
 
 
@@ -679,6 +808,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=C2.name, choices=sorted(k for k, v in WORKLOADS.items() if hasattr(v, "L")))
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the 128K fwd+bwd leg")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch fwd+bwd leg")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-blocks", type=int, default=16)

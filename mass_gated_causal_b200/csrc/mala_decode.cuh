@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(misc + 0);
   uint32_t* sflag = misc + 1;  // bit 0: some head keeps the tile; bit 1: abort
+  int* sPage = reinterpret_cast<int*>(misc + 4);  // [8] paged cache: page of tile t at t & 7, set by the producer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int nbk = p.B * p.Hkv;
@@ -167,20 +168,13 @@ __global__ void __launch_bounds__(320, 1)
   const int t1 = bad ? nk : min(t0 + tps, nk);
   const int T = t1 - t0;  // tiles kb = t1-1 ... t0
   const FailState fs{abort_flag, p.status};
-  // TMA coordinates (row, outer index) of key tile kb: a page of the pool, or rows of sequence b
-  auto tile_at = [&](int kb, int& row, int& outer) {
-    if (kPaged) {
-      const int pg = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + kb);
-      row = 0;
-      outer = pg;
-      if (pg < 0 || pg >= p.num_pages) {  // read as zeros (a load outside the tensor fills), reported
-        atomicOr(p.status, kStatusSeqTable);
-        outer = p.num_pages;
-      }
-    } else {
-      row = kb * BK;
-      outer = b;
-    }
+  // paged cache: the page of key tile kb, checked (an id outside the pool is
+  // reported and read as zeros: a TMA load outside the tensor fills)
+  auto page_of = [&](int kb) {
+    const int pg = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + kb);
+    if (pg >= 0 && pg < p.num_pages) return pg;
+    atomicOr(p.status, kStatusSeqTable);
+    return p.num_pages;
   };
   if (bad && sp_idx == 0 && tid == 0) atomicOr(p.status, kStatusSeqTable);
 
@@ -217,11 +211,14 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
+      int pg_next = kPaged ? page_of(t1 - 1) : 0;  // page ids are read a tile ahead
       for (int t = 0; t < T; ++t) {
         const int st = t % NK;
+        const int pg = pg_next;
+        if (kPaged && t + 1 < T) pg_next = page_of(t1 - 2 - t);
         if (t >= NK && !mbar_wait(&k_empty[st], ((t / NK) - 1) & 1, fs)) break;
-        int krow, kouter;
-        tile_at(t1 - 1 - t, krow, kouter);
+        const int krow = kPaged ? 0 : (t1 - 1 - t) * BK, kouter = kPaged ? pg : b;
+        if (kPaged) sPage[t & 7] = pg;  // for the gate warp's V request (it trails by < 8 tiles)
         mbar_arrive_expect_tx(&k_full[st], TB);
         for (int h = 0; h < D / 64; ++h)
           tma_load_4d(&tm_k, &k_full[st], sK + st * TB + h * (BK * 128), h * 64, hkv, krow, kouter);
@@ -275,8 +272,7 @@ __global__ void __launch_bounds__(320, 1)
         const bool ab = abort_raised(fs);
         if (any && !ab) {  // V is requested only now that a head keeps the tile
           const int vs = nkept % NV;
-          int vrow, vouter;
-          tile_at(kb, vrow, vouter);
+          const int vrow = kPaged ? 0 : kb * BK, vouter = kPaged ? sPage[t & 7] : b;
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(&v_full[vs], TB);
           for (int h = 0; h < D / 64; ++h)

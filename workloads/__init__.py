@@ -148,6 +148,39 @@ C3 = TrainWorkload("mala_fwd_bwd_L128k_h8_d128", 1, 8, 8, 131072, 128, 128, 128,
 C4 = DecodeWorkload("mala_decode_B8_Lk128k_gqa32x8_d128", 8, 32, 8, 131072, 128, 128, seed=1004, taus=(1.0, 0.0))
 
 WORKLOADS = {w.name: w for w in (C0, C1, C1_IID, C2, C3, C4)}
+
+
+@dataclass(frozen=True)
+class PackedWorkload:
+    """A packed batch of training sequences laid end to end (lengths `lens`)."""
+    name: str
+    lens: tuple
+    Hq: int
+    Hkv: int
+    d: int
+    Bq: int
+    Bk: int
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def total(self) -> int:
+        return int(sum(self.lens))
+
+    def describe(self) -> dict:
+        out = asdict(self)
+        out["scale"] = self.scale
+        out["total"] = self.total
+        return out
+
+
+# A 32K-token packed batch: nine sequences of mixed, mostly ragged lengths
+# (a long document down to a short one), GQA 32/8 as in the 32K workload.
+C5 = PackedWorkload("mala_fwd_bwd_varlen_T32k_gqa32x8_d128",
+                    (12000, 7300, 4100, 3000, 2600, 1500, 1111, 700, 457), 32, 8, 128, 128, 128, seed=1005)
 SUBSET_SEED_OFFSET = 500
 
 
@@ -250,6 +283,21 @@ def make_train_inputs(w: TrainWorkload, workers: int = 1, seed: Optional[int] = 
         for j in jobs:
             _store(_train_kv_job(j))
     return {"q": q, "k": k, "v": v, "do": do}
+
+
+def make_packed_inputs(w: PackedWorkload, workers: int = 1):
+    """bf16 bit tensors of a packed batch: q, dO [total, Hq, d], k, v [total, Hkv, d]
+    (uint16) and cu_seqlens [S + 1] (int32). Sequence s is the training recipe for
+    one sequence of length lens[s] with seed w.seed * 100 + s."""
+    parts = {"q": [], "k": [], "v": [], "do": []}
+    for s, L in enumerate(w.lens):
+        t = make_train_inputs(TrainWorkload(w.name, 1, w.Hq, w.Hkv, int(L), w.d, w.Bq, w.Bk, seed=w.seed * 100 + s),
+                              workers=workers)
+        for x in parts:
+            parts[x].append(t[x][0])
+    out = {x: np.concatenate(v, 0) for x, v in parts.items()}
+    out["cu_seqlens"] = np.concatenate([[0], np.cumsum(w.lens)]).astype(np.int32)
+    return out
 
 
 def _decode_kv_job(args):
