@@ -631,6 +631,53 @@ def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_rank
     out["mala_speedup"] = round(out["tau0"]["us_per_step"] / out["tau1"]["us_per_step"], 3)
     out["hbm_peak_gbs"] = pk["hbm_gbs"]
     out["paged"] = run_paged_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, out)
+    out["exact"] = run_exact_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, out)
+    return out
+
+
+def run_exact_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, contiguous):
+    """mala_decode_exact on the decode workload: the single-pass decisions, the
+    same split count for the PV work. Algorithmic bytes as for mala_decode (K,
+    V of the kept tiles, q, o); the fp32 scores it writes and reads back are
+    reported beside them."""
+    B, Hq, d = q.shape
+    Lk, Hkv = kc.shape[1], kc.shape[2]
+    ns = contiguous["n_splits"]
+    nk = -(-Lk // w.Bk)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    kept = torch.empty((B * Hq,), dtype=torch.int32, device=dev)
+    wsb = mala.mala_decode_exact_workspace_size(B, Hq, Lk, d, w.Bk, ns)
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+    aux = 2 * B * Hq * nk * w.Bk * 4  # scores written once, read once
+    out = {"workload": w.name + "_exact", "n_splits": ns, "scores_bytes_per_step": aux}
+    for tau in (1.0, 0.0):
+        km = torch.zeros((B, Hq, nk), dtype=torch.uint8, device=dev)
+        rc = mala.mala_decode_exact(q, kc, vc, o, lse, B, Hq, Hkv, Lk, d, w.scale, tau, w.Bk, ns, ws, wsb, kept, km,
+                                    stream)
+        assert rc == 0
+        assert mala.mala_check_status(stream) == 0
+        kmh = km.cpu().numpy()
+        by = decode_bytes(B, Hq, Hkv, Lk, d, w.Bk, kmh)
+        del km
+
+        def fn(mid=None, tau_=tau):
+            rc_ = mala.mala_decode_exact(q, kc, vc, o, lse, B, Hq, Hkv, Lk, d, w.scale, tau_, w.Bk, ns, ws, wsb, kept,
+                                         None, stream)
+            assert rc_ == 0
+            if mid is not None:
+                mid.record(stream)
+        tot, _, _ = timed(fn, max(5, args.steps * 2), max(3, args.warmup))
+        us = max_over_ranks(float(np.median(tot))) * 1e3
+        gbs = by["total"] / (us * 1e-6) / 1e9
+        key = f"tau{int(tau)}"
+        out[key] = {"us_per_step": round(us, 1), "us_per_token": round(us / B, 2), "GBps": round(gbs, 1),
+                    "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
+                    "frac_of_hbm_with_scores": round((by["total"] + aux) / (us * 1e-6) / 1e9 / pk["hbm_gbs"], 4),
+                    "bytes_per_step": by["total"], "v_tile_frac": round(by["v_tile_frac"], 4),
+                    "retained_tile_frac_per_head": round(float((kmh == 1).mean()), 4),
+                    "vs_split_decode": round(contiguous[key]["us_per_step"] / us, 3)}
+    assert mala.mala_check_status(stream) == 0
     return out
 
 

@@ -277,6 +277,41 @@ MALA_API int mala_decode(const void* q, const void* kcache, const void* vcache, 
                 void* stream);
 
 /*
+ * Workspace bytes mala_decode_exact needs: fp32 scores [B, Hq, nk * Bk], per
+ * tile (max, log-sum) pairs [B, Hq, nk], decisions [B, Hq, nk] and the split
+ * partials of mala_decode_workspace_size, each 256-byte aligned. 0 for
+ * invalid sizes.
+ */
+MALA_API size_t mala_decode_exact_workspace_size(int B, int Hq, int Lk, int d, int Bk, int n_splits);
+
+/*
+ * mala_decode_exact -- decode whose decisions do not depend on the split.
+ *
+ * Source: agihunt.info MALA digest, method paragraphs (the forward gate: tiles
+ * from the newest to the oldest against the state over the kept tiles, the
+ * first tile kept).
+ *
+ * The decisions are those of ONE sequential pass over all nk tiles (exactly
+ * mala_decode with n_splits = 1, i.e. the forward's last query row): tile t
+ * is kept iff it is the newest, or tau == 0, or 2^{M_t} / Z >= tau / Lk with
+ * M_t its largest score and Z the sum of exp over the kept newer tiles (log2
+ * units inside). The work runs in three phases: every score and each tile's
+ * (max, log-sum) pair (K read once), a per-row scan of the decisions over
+ * those pairs, and the PV of the kept tiles split over n_splits ranges of
+ * tiles per (b, KV head) with the usual merge by LSE. n_splits only spreads
+ * the PV work; it does not change any decision. V is read only for tiles some
+ * head of the group keeps; the scores cost 8 extra bytes per key and head
+ * (written once, read once).
+ *
+ * Arguments and layouts as mala_decode; workspace >=
+ * mala_decode_exact_workspace_size(B, Hq, Lk, d, Bk, n_splits used) bytes.
+ * kept_tiles [B*Hq] and keep_map [B, Hq, nk] (nullable) hold the decisions.
+ */
+MALA_API int mala_decode_exact(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B,
+             int Hq, int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, void* workspace,
+             size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
+
+/*
  * mala_decode_paged -- mala_decode against a paged KV cache.
  *
  * Source: as mala_decode (the cache is kept whole; decode reads it).

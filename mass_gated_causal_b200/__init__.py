@@ -38,6 +38,7 @@ MALA_ERR_RANGE = 6
 EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_prefill", "mala_fwd_varlen",
             "mala_fwd_workspace_size", "mala_bwd_workspace_size", "mala_bwd", "mala_bwd_varlen",
             "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_paged",
+            "mala_decode_exact_workspace_size", "mala_decode_exact",
             "mala_decode_noalloc_max_bytes", "mala_decode_noalloc", "mala_check_status")
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -58,6 +59,11 @@ _lib.mala_bwd_varlen.restype = _i
 _lib.mala_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _i, _vp,
                                    _sz, _vp, _vp, _vp]
 _lib.mala_decode_paged.restype = _i
+_lib.mala_decode_exact_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
+_lib.mala_decode_exact_workspace_size.restype = _sz
+_lib.mala_decode_exact.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp,
+                                   _vp]
+_lib.mala_decode_exact.restype = _i
 _lib.mala_fwd_workspace_size.argtypes = [_i, _i, _i, _i]
 _lib.mala_fwd_workspace_size.restype = _sz
 _lib.mala_bwd_workspace_size.argtypes = [_i, _i, _i, _i]
@@ -185,6 +191,17 @@ def mala_decode(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_
     return int(_lib.mala_decode(_p(q), _p(kcache), _p(vcache), _p(o), _p(lse), B, Hq, Hkv, Lk, d, float(scale),
                                 float(tau), Bk, n_splits, _p(workspace), int(workspace_bytes), _p(kept_tiles),
                                 _p(keep_map), _stream(stream)))
+
+
+def mala_decode_exact_workspace_size(B, Hq, Lk, d, Bk, n_splits) -> int:
+    return int(_lib.mala_decode_exact_workspace_size(B, Hq, Lk, d, Bk, n_splits))
+
+
+def mala_decode_exact(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, workspace,
+                      workspace_bytes, kept_tiles, keep_map=None, stream=None) -> int:
+    return int(_lib.mala_decode_exact(_p(q), _p(kcache), _p(vcache), _p(o), _p(lse), B, Hq, Hkv, Lk, d,
+                                      float(scale), float(tau), Bk, n_splits, _p(workspace), int(workspace_bytes),
+                                      _p(kept_tiles), _p(keep_map), _stream(stream)))
 
 
 def mala_decode_noalloc_max_bytes() -> int:
@@ -349,4 +366,24 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens_k, scale: float, tau:
     _check(mala_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, o, lse, B, Hq, Hkv, num_pages, page, maxp,
                              d, scale, tau, n_splits, workspace, workspace.numel() * workspace.element_size(), kept,
                              km, stream), "mala_decode_paged")
+    return o, lse, kept, km, n_splits
+
+
+def decode_exact(q, kcache, vcache, scale: float, tau: float, Bk: int = 128, n_splits: int = 0,
+                 keep_map: bool = False, workspace=None, stream=None):
+    """Split-independent decode -> (o, lse, kept_tiles, keep_map|None, n_splits)."""
+    import torch
+    B, Hq, d = q.shape
+    Lk, Hkv = kcache.shape[1], kcache.shape[2]
+    if n_splits == 0:
+        n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    kept = torch.empty((B * Hq,), dtype=torch.int32, device=q.device)
+    ws_bytes = mala_decode_exact_workspace_size(B, Hq, Lk, d, Bk, n_splits)
+    if workspace is None:
+        workspace = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device=q.device)
+    km = torch.full((B, Hq, -(-Lk // Bk)), 255, dtype=torch.uint8, device=q.device) if keep_map else None
+    _check(mala_decode_exact(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, workspace,
+                             workspace.numel() * workspace.element_size(), kept, km, stream), "mala_decode_exact")
     return o, lse, kept, km, n_splits

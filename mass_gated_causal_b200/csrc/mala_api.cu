@@ -17,6 +17,7 @@
 #include "../../include/mala.h"
 #include "mala_bwd.cuh"
 #include "mala_decode.cuh"
+#include "mala_decode_exact.cuh"
 #include "mala_fwd.cuh"
 
 namespace {
@@ -210,6 +211,31 @@ int launch_dec_gate(bool gate, const CUtensorMap& mk, const CUtensorMap& mv, con
                     cudaStream_t st) {
   return gate ? launch_dec_g<D, BK, true>(mk, mv, p, st) : launch_dec_g<D, BK, false>(mk, mv, p, st);
 }
+
+template <int D, int BK, int GP>
+int launch_dx(const mala::DxParams& p, cudaStream_t st) {
+  const unsigned g1 = static_cast<unsigned>(p.B) * p.Hkv * ((p.nk + 7) / 8);
+  mala::mala_dx_scores_kernel<D, BK, GP><<<g1, 256, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
+  mala::mala_dx_scan_kernel<<<(p.B * p.Hq + 3) / 4, 128, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
+  const unsigned g3 = static_cast<unsigned>(p.B) * p.Hkv * p.n_splits;
+  mala::mala_dx_pv_kernel<D, BK, GP><<<g3, 256, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
+  mala::mala_decode_combine_kernel<D><<<(p.B * p.Hq + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
+                                                                         reinterpret_cast<uint16_t*>(p.o_out),
+                                                                         p.lse_out, p.B * p.Hq, p.n_splits);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
+template <int D, int BK>
+int launch_dx_g(const mala::DxParams& p, cudaStream_t st) {
+  if (p.G <= 1) return launch_dx<D, BK, 1>(p, st);
+  if (p.G <= 2) return launch_dx<D, BK, 2>(p, st);
+  if (p.G <= 4) return launch_dx<D, BK, 4>(p, st);
+  return launch_dx<D, BK, 8>(p, st);
+}
+
 
 }  // namespace
 
@@ -589,6 +615,68 @@ int mala_decode_paged(const void* q, const void* k_pages, const void* v_pages, c
   pg.num_pages = num_pages;
   return run_decode(q, mk, mv, o, lse, B, Hq, Hkv, static_cast<int>(max_lk), d, scale, tau, page_size, n_splits,
                     workspace, kept_tiles, keep_map, static_cast<cudaStream_t>(stream), pg);
+}
+
+namespace {
+struct DxWorkspace {
+  size_t scores, tile_ml, keep, o_part, lse_part, total;
+};
+
+DxWorkspace dx_layout(int B, int Hq, int Lk, int d, int Bk, int n_splits) {
+  DxWorkspace w;
+  const size_t nk = (static_cast<size_t>(Lk) + Bk - 1) / Bk;
+  const size_t rows = static_cast<size_t>(B) * Hq;
+  w.scores = 0;
+  w.tile_ml = w.scores + align256(rows * nk * Bk * 4);
+  w.keep = w.tile_ml + align256(rows * nk * 8);
+  w.o_part = w.keep + align256(rows * nk);
+  w.lse_part = w.o_part + align256(rows * n_splits * d * 4);
+  w.total = w.lse_part + align256(rows * n_splits * 4);
+  return w;
+}
+}  // namespace
+
+size_t mala_decode_exact_workspace_size(int B, int Hq, int Lk, int d, int Bk, int n_splits) {
+  if (B < 1 || Hq < 1 || Lk < 1 || n_splits < 1 || (d != 64 && d != 128) || (Bk != 64 && Bk != 128)) return 0;
+  return dx_layout(B, Hq, Lk, d, Bk, n_splits).total;
+}
+
+int mala_decode_exact(const void* q, const void* kcache, const void* vcache, void* o, float* lse, int B, int Hq,
+                      int Hkv, int Lk, int d, float scale, float tau, int Bk, int n_splits, void* workspace,
+                      size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream) {
+  int rc = check_decode_args(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau, Bk, n_splits, kept_tiles);
+  if (rc != MALA_OK) return rc;
+  if (n_splits == 0) n_splits = mala_decode_default_splits(B, Hkv, Lk, Bk);
+  if (n_splits > 65535) return MALA_ERR_UNSUPPORTED;
+  const DxWorkspace lay = dx_layout(B, Hq, Lk, d, Bk, n_splits);
+  if (!workspace || workspace_bytes < lay.total || !aligned256(workspace)) return MALA_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  mala::DxParams p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.Lk = Lk;
+  p.nk = (Lk + Bk - 1) / Bk;
+  p.n_splits = n_splits;
+  p.tiles_per_split = (p.nk + n_splits - 1) / n_splits;
+  p.Lkp = p.nk * Bk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.gate = tau > 0.f ? 1 : 0;
+  p.thr = tau > 0.f ? std::log2(tau) - std::log2(static_cast<float>(Lk)) : 0.f;
+  p.q = static_cast<const uint16_t*>(q);
+  p.kc = static_cast<const uint16_t*>(kcache);
+  p.vc = static_cast<const uint16_t*>(vcache);
+  p.scores = reinterpret_cast<float*>(ws + lay.scores);
+  p.tile_ml = reinterpret_cast<float2*>(ws + lay.tile_ml);
+  p.keep = reinterpret_cast<uint8_t*>(ws + lay.keep);
+  p.o_part = reinterpret_cast<float*>(ws + lay.o_part);
+  p.lse_part = reinterpret_cast<float*>(ws + lay.lse_part);
+  p.kept_tiles = kept_tiles;
+  p.keep_map = keep_map;
+  p.o_out = o;
+  p.lse_out = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128 && Bk == 128) return launch_dx_g<128, 128>(p, st);
+  if (d == 64 && Bk == 128) return launch_dx_g<64, 128>(p, st);
+  if (d == 128 && Bk == 64) return launch_dx_g<128, 64>(p, st);
+  return launch_dx_g<64, 64>(p, st);
 }
 
 int mala_check_status(void* stream) {

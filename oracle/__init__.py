@@ -365,3 +365,11 @@ def paged_decode(q, k_pages, v_pages, block_table, seqlens, scale: float, tau: f
             margin[b, hq, :npg] = r["margin"][0, hq]
             kept[b * Hq + hq] = r["kept"][hq]
     return {"o": o, "lse": lse, "keep": keep, "margin": margin, "kept": kept}
+
+
+def decode_single_pass(q, kc, vc, scale: float, tau: float, Bk: int, sel: Optional[Sequence] = None):
+    """Decode as ONE sequential pass over all key tiles (newest to oldest, the
+    first kept): ``decode`` with a single split, which equals the forward's last
+    query row (pinned in tests/test_oracle.py). A split-independent decode must
+    reach exactly these decisions whatever split of the tiles it uses."""
+    return decode(q, kc, vc, scale, tau, Bk, 1, sel=sel)

@@ -179,6 +179,33 @@ def test_decode_rejects(kw, code):
     assert dec(**kw) == code
 
 
+def dex(**kw):
+    a = dict(q=P, kcache=P, vcache=P, o=P, lse=P, B=2, Hq=8, Hkv=2, Lk=1000, d=128, scale=0.1, tau=1.0, Bk=128,
+             n_splits=4, workspace=P, workspace_bytes=1 << 30, kept_tiles=P, keep_map=None, stream=S)
+    a.update(kw)
+    return mala.mala_decode_exact(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(Hq=6, Hkv=4), 1), (dict(n_splits=-1), 1), (dict(tau=-0.5), 1),
+    (dict(d=32), 2), (dict(Bk=256), 2), (dict(Hq=32, Hkv=2), 2), (dict(vcache=P + 2), 2),
+    (dict(workspace=None), 3), (dict(workspace_bytes=1000), 3), (dict(workspace=P + 32), 3),
+])
+def test_decode_exact_rejects(kw, code):
+    assert dex(**kw) == code
+
+
+def test_decode_exact_workspace_size():
+    a256 = lambda x: (x + 255) // 256 * 256
+    B, Hq, Lk, d, Bk, S = 2, 8, 1000, 128, 128, 5
+    nk = -(-Lk // Bk)
+    want = a256(B * Hq * nk * Bk * 4) + a256(B * Hq * nk * 8) + a256(B * Hq * nk) + a256(B * Hq * S * d * 4) + \
+        a256(B * Hq * S * 4)
+    assert mala.mala_decode_exact_workspace_size(B, Hq, Lk, d, Bk, S) == want
+    assert mala.mala_decode_exact_workspace_size(B, Hq, Lk, d, 96, S) == 0
+    assert mala.mala_decode_exact_workspace_size(B, Hq, Lk, d, Bk, 0) == 0
+
+
 def test_decode_sizes_and_default_splits():
     a256 = lambda x: (x + 255) // 256 * 256
     assert mala.mala_decode_workspace_size(2, 8, 128, 5) == a256(2 * 8 * 5 * 128 * 4) + a256(2 * 8 * 5 * 4)
