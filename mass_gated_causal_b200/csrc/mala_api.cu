@@ -213,14 +213,17 @@ int launch_dec_gate(bool gate, const CUtensorMap& mk, const CUtensorMap& mv, con
 }
 
 template <int D, int BK, int GP>
-int launch_dx(const mala::DxParams& p, cudaStream_t st) {
+int launch_dx(const CUtensorMap& mv, const mala::DxParams& p, cudaStream_t st) {
+  using Lay = mala::DxLayout<D, BK, GP>;
+  auto kpv = mala::mala_dx_pv_kernel<D, BK, GP>;
+  if (set_smem(kpv, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned g1 = static_cast<unsigned>(p.B) * p.Hkv * ((p.nk + 7) / 8);
   mala::mala_dx_scores_kernel<D, BK, GP><<<g1, 256, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
   mala::mala_dx_scan_kernel<<<(p.B * p.Hq + 3) / 4, 128, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
   const unsigned g3 = static_cast<unsigned>(p.B) * p.Hkv * p.n_splits;
-  mala::mala_dx_pv_kernel<D, BK, GP><<<g3, 256, 0, st>>>(p);
+  kpv<<<g3, 288, Lay::ALLOC_BYTES, st>>>(mv, p);
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
   mala::mala_decode_combine_kernel<D><<<(p.B * p.Hq + 3) / 4, 128, 0, st>>>(p.o_part, p.lse_part,
                                                                          reinterpret_cast<uint16_t*>(p.o_out),
@@ -229,11 +232,11 @@ int launch_dx(const mala::DxParams& p, cudaStream_t st) {
 }
 
 template <int D, int BK>
-int launch_dx_g(const mala::DxParams& p, cudaStream_t st) {
-  if (p.G <= 1) return launch_dx<D, BK, 1>(p, st);
-  if (p.G <= 2) return launch_dx<D, BK, 2>(p, st);
-  if (p.G <= 4) return launch_dx<D, BK, 4>(p, st);
-  return launch_dx<D, BK, 8>(p, st);
+int launch_dx_g(const CUtensorMap& mv, const mala::DxParams& p, cudaStream_t st) {
+  if (p.G <= 1) return launch_dx<D, BK, 1>(mv, p, st);
+  if (p.G <= 2) return launch_dx<D, BK, 2>(mv, p, st);
+  if (p.G <= 4) return launch_dx<D, BK, 4>(mv, p, st);
+  return launch_dx<D, BK, 8>(mv, p, st);
 }
 
 
@@ -672,11 +675,16 @@ int mala_decode_exact(const void* q, const void* kcache, const void* vcache, voi
   p.keep_map = keep_map;
   p.o_out = o;
   p.lse_out = lse;
+  unsigned* status = status_ptr();
+  if (!status) return MALA_ERR_CUDA;
+  p.status = status;
+  CUtensorMap mv;
+  if (!make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk)) return MALA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128 && Bk == 128) return launch_dx_g<128, 128>(p, st);
-  if (d == 64 && Bk == 128) return launch_dx_g<64, 128>(p, st);
-  if (d == 128 && Bk == 64) return launch_dx_g<128, 64>(p, st);
-  return launch_dx_g<64, 64>(p, st);
+  if (d == 128 && Bk == 128) return launch_dx_g<128, 128>(mv, p, st);
+  if (d == 64 && Bk == 128) return launch_dx_g<64, 128>(mv, p, st);
+  if (d == 128 && Bk == 64) return launch_dx_g<128, 64>(mv, p, st);
+  return launch_dx_g<64, 64>(mv, p, st);
 }
 
 int mala_check_status(void* stream) {

@@ -14,15 +14,18 @@
 //   mala_dx_scores_kernel  every score s = scale * log2(e) * <q, k> of every
 //                          query head, stored (fp32), and (M_t, L_t) per tile
 //                          and head; K is read once, by the G heads of a group
-//                          together
+//                          together, a warp per tile (many warps per SM keep the
+//                          loads in flight; a TMA-ring version measured slower)
 //   mala_dx_scan_kernel    one warp per (b, query head) walks the chain 32
 //                          tiles at a time: it assumes the 32 tiles' decisions,
-//                          forms every tile's Z_prev with a log-add-exp scan,
-//                          and corrects the first wrong assumption until none
-//                          is left (each round fixes at least one tile)
+//                          forms every tile's Z_prev with a prefix sum (linear
+//                          units relative to the chunk's largest log-sum), and
+//                          corrects the first wrong assumption until none is
+//                          left (each round fixes at least one tile)
 //   mala_dx_pv_kernel      per (b, KV head, split of the tiles): P = 2^{s - m}
 //                          on the kept tiles and P V, the split's O and LSE; V
-//                          is read only for tiles some head of the group keeps
+//                          of the tiles some head of the group keeps streams in
+//                          by TMA through a ring, and no other V is read
 // and mala_decode_combine_kernel merges the splits by their LSEs.
 #pragma once
 
@@ -48,13 +51,32 @@ struct DxParams {
   uint8_t* keep_map;    // [B, Hq, nk], nullable
   void* o_out;          // [B, Hq, d] bf16 (written by the merge)
   float* lse_out;       // [B, Hq]
+  unsigned* status;
 };
 
-// log2(2^a + 2^b), with -inf as the empty sum
-__device__ __forceinline__ float lae2(float a, float b) {
-  const float hi = fmaxf(a, b), lo = fminf(a, b);
-  if (lo == -INFINITY) return hi;
-  return hi + lg2_approx(1.f + ex2_approx(lo - hi));
+// Shared-memory layout of the PV kernel: an NS-stage ring of
+// [D/64][BK][64] bf16 tiles (128-byte swizzle, as the TMA writes them), a
+// [2][GP][BK] fp32 tile and the ring's barriers.
+template <int D, int BK, int GP>
+struct DxLayout {
+  static constexpr int NS = 4;
+  static constexpr int TB = BK * D * 2;
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_T = OFF_RING + NS * TB;        // fp32 [2][GP][BK]: P by tile parity
+  static constexpr int OFF_O = OFF_T + 2 * GP * BK * 4;   // fp32 [8][GP][D + 4] (PV reduction)
+  static constexpr int OFF_LIST = OFF_O + 8 * GP * (D + 4) * 4;  // int tiles [LIST], uint8 bits [LIST]
+  static constexpr int LIST = 1024;
+  static constexpr int OFF_BAR = (OFF_LIST + LIST * 5 + 7) & ~7;
+  static constexpr int OFF_MISC = OFF_BAR + 2 * NS * 8;
+  static constexpr int BYTES = OFF_MISC + 128;  // abort flag, list count, m and l per head
+  static constexpr int ALLOC_BYTES = BYTES + 1024;
+  static_assert(ALLOC_BYTES <= 232448, "shared memory exceeds the per-CTA limit");
+};
+
+// 16-byte chunk cc of row j of a [D/64][BK][64] bf16 tile with 128-byte swizzle
+template <int BK>
+__device__ __forceinline__ uint32_t dx_row_chunk(uint32_t base, int j, int cc) {
+  return base + (cc >> 3) * (BK * 128) + j * 128 + (((cc & 7) ^ (j & 7)) << 4);
 }
 
 // ---------------------------------------------------------------- scores
@@ -84,9 +106,9 @@ __global__ void __launch_bounds__(256) mala_dx_scores_kernel(const DxParams p) {
       qf[g][e] = g < p.G ? bf16lo_to_f32(p.q[(static_cast<size_t>(b) * p.Hq + hq0 + g) * D + c * CPL + e]) : 0.f;
   const uint16_t* krow0 = p.kc + (static_cast<size_t>(b) * p.Lk * p.Hkv + hkv) * D + c * CPL;
   const size_t kstride = static_cast<size_t>(p.Hkv) * D;
-  constexpr int UNR = 4;
-  for (int it0 = 0; it0 < BK / 2; it0 += UNR) {
-    uint32_t raw[UNR][CPL / 2];
+  constexpr int UNR = 4;  // rows per lane and group; the next group's loads are issued before this one is used
+  uint32_t nxt[UNR][CPL / 2];
+  auto load_group = [&](int it0) {
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
       const int j = kb * BK + (it0 + u) * 2 + half;
@@ -94,16 +116,25 @@ __global__ void __launch_bounds__(256) mala_dx_scores_kernel(const DxParams p) {
         const uint16_t* src = krow0 + static_cast<size_t>(j) * kstride;
         if constexpr (CPL == 8) {
           const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
-          raw[u][0] = v.x; raw[u][1] = v.y; raw[u][2] = v.z; raw[u][3] = v.w;
+          nxt[u][0] = v.x; nxt[u][1] = v.y; nxt[u][2] = v.z; nxt[u][3] = v.w;
         } else {
           const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-          raw[u][0] = v.x; raw[u][1] = v.y;
+          nxt[u][0] = v.x; nxt[u][1] = v.y;
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < CPL / 2; ++e) raw[u][e] = 0u;
+        for (int e = 0; e < CPL / 2; ++e) nxt[u][e] = 0u;
       }
     }
+  };
+  load_group(0);
+  for (int it0 = 0; it0 < BK / 2; it0 += UNR) {
+    uint32_t raw[UNR][CPL / 2];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u)
+#pragma unroll
+      for (int e = 0; e < CPL / 2; ++e) raw[u][e] = nxt[u][e];
+    if (it0 + UNR < BK / 2) load_group(it0 + UNR);
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
       float part[GP];
@@ -170,26 +201,35 @@ __global__ void __launch_bounds__(128) mala_dx_scan_kernel(const DxParams p) {
     const bool valid = t < p.nk;
     const int kb = p.nk - 1 - t;
     const float2 v = valid ? ml[kb] : make_float2(-INFINITY, -INFINITY);
+    // linear units relative to R, the largest log-sum in play: every term <= 1,
+    // so the rounds below are plain sums and compares
+    float R = fmaxf(logZ, v.y);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) R = fmaxf(R, __shfl_xor_sync(0xffffffffu, R, o));
+    if (R == -INFINITY) R = 0.f;
+    const float zl = logZ == -INFINITY ? 0.f : ex2_approx(logZ - R);  // the kept tiles before this chunk
+    const float w = valid ? ex2_approx(v.y - R) : 0.f;                 // my tile's sum
+    const float e = valid ? ex2_approx(v.x - p.thr - R) : 0.f;         // 2^{M - thr}: keep iff e >= Z_prev
     bool tent = valid;  // assumed decision
-    float incl = -INFINITY;
+    float incl = 0.f;
     for (int round = 0; round <= 32; ++round) {
-      // Z of the assumed kept tiles before me in this chunk (log-add-exp scan)
-      incl = tent ? v.y : -INFINITY;
+      // Z of the assumed kept tiles before me in this chunk (prefix sum)
+      incl = tent ? w : 0.f;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl = lae2(incl, u);
+        if (lane >= o) incl += u;
       }
       float excl = __shfl_up_sync(0xffffffffu, incl, 1);
-      if (lane == 0) excl = -INFINITY;
-      const float zprev = lae2(logZ, excl);
-      const bool dec = valid && (t == 0 || !p.gate || v.x - zprev >= p.thr);  // ties keep
+      if (lane == 0) excl = 0.f;
+      const bool dec = valid && (t == 0 || !p.gate || e >= zl + excl);  // ties keep
       const unsigned mism = __ballot_sync(0xffffffffu, dec != tent);
       if (mism == 0u) break;
       const int f = __ffs(mism) - 1;  // every tile before f was assumed right, so f's decision is right
       if (lane >= f) tent = dec;      // f is now final; later tiles take a fresh guess
     }
-    logZ = lae2(logZ, __shfl_sync(0xffffffffu, incl, 31));
+    const float zt = zl + __shfl_sync(0xffffffffu, incl, 31);
+    if (zt > 0.f) logZ = R + lg2_approx(zt);
     if (valid) {
       kp[kb] = tent ? 1 : 0;
       if (p.keep_map) p.keep_map[static_cast<size_t>(row) * p.nk + kb] = tent ? 1 : 0;
@@ -200,20 +240,36 @@ __global__ void __launch_bounds__(128) mala_dx_scan_kernel(const DxParams p) {
 }
 
 // ---------------------------------------------------------------- PV
-// One CTA of 8 warps per (b, KV head, split). Per head the split's offset m is
-// the largest M_t of its kept tiles and its normaliser l = sum over those tiles
-// of 2^{L_t - m} (both from the per-tile pairs). A tile some head keeps is read
-// once: its P = 2^{s - m} (0 for a head that skips it) goes to shared memory,
-// and warp w takes keys [BK/8 * w, BK/8 * (w+1)), two per step: lane c of half
-// h accumulates D/16 columns of the G heads' P V over its rows.
+// One CTA per (b, KV head, split). Per head the split's offset m is the
+// largest M_t of its kept tiles and its normaliser l = sum over those tiles of
+// 2^{L_t - m} (both from the per-tile pairs). Warp 8 lists the tiles some head
+// of the group keeps (with a bit per head) and streams their V by TMA through
+// the ring; a tile no head keeps is never read. Per listed tile the compute
+// warps form P = 2^{s - m} (0 for a head that skips the tile; the scores of
+// the next tile are loaded while this one is used) in shared memory, and warp
+// w takes keys [BK/8 * w, BK/8 * (w+1)), two per step: lane c of half h
+// accumulates D/16 columns of the G heads' P V over its rows.
 template <int D, int BK, int GP>
-__global__ void __launch_bounds__(256) mala_dx_pv_kernel(const DxParams p) {
+__global__ void __launch_bounds__(288, 1) mala_dx_pv_kernel(const __grid_constant__ CUtensorMap tm_v,
+                                                              const DxParams p) {
+  using Lay = DxLayout<D, BK, GP>;
+  constexpr int NS = Lay::NS, TB = Lay::TB, LIST = Lay::LIST;
   constexpr int CPL = D / 16;
-  constexpr int KPW = BK / 8;  // keys per warp and tile
-  __shared__ float sP[GP][BK];
-  __shared__ float sM[GP], sLn[GP];
-  __shared__ int sKeep[2][GP];  // by tile parity: a skipped tile's flags may still be read
-  __shared__ float sO[8][GP][D + 4];
+  constexpr int KPW = BK / 8;                   // keys per compute warp and tile
+  constexpr int NPT = (GP * BK + 255) / 256;    // P entries per compute thread
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* sP = reinterpret_cast<float*>(smem + Lay::OFF_T);  // [2][GP][BK]
+  float* sO = reinterpret_cast<float*>(smem + Lay::OFF_O);  // [8][GP][D + 4]
+  int* sList = reinterpret_cast<int*>(smem + Lay::OFF_LIST);
+  uint8_t* sBits = smem + Lay::OFF_LIST + LIST * 4;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* empty = full + NS;
+  int* misc = reinterpret_cast<int*>(smem + Lay::OFF_MISC);
+  int* abort_flag = misc;
+  int* sCount = misc + 1;
+  float* sM = reinterpret_cast<float*>(misc + 2);  // [GP]
+  float* sLn = sM + GP;                            // [GP]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int nbk = p.B * p.Hkv;
   const int bk = blockIdx.x % nbk, sp = blockIdx.x / nbk;
@@ -221,7 +277,11 @@ __global__ void __launch_bounds__(256) mala_dx_pv_kernel(const DxParams p) {
   const int hq0 = hkv * p.G;
   const size_t r0 = static_cast<size_t>(b) * p.Hq + hq0;  // row of head 0 of the group
   const int t0 = min(sp * p.tiles_per_split, p.nk), t1 = min(t0 + p.tiles_per_split, p.nk);
-  const int c = lane & 15, half = lane >> 4;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 8); }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
   if (warp < GP) {  // warp g: the offset and normaliser of head g over this split
     float m = -INFINITY;
     if (warp < p.G)
@@ -240,79 +300,127 @@ __global__ void __launch_bounds__(256) mala_dx_pv_kernel(const DxParams p) {
       sLn[warp] = l;
     }
   }
+  __syncthreads();
+  const FailState fs{abort_flag, p.status};
+  const int c = lane & 15, half = lane >> 4;
   float acc[GP][CPL];
 #pragma unroll
   for (int g = 0; g < GP; ++g)
 #pragma unroll
     for (int e = 0; e < CPL; ++e) acc[g][e] = 0.f;
-  const uint16_t* vrow0 = p.vc + (static_cast<size_t>(b) * p.Lk * p.Hkv + hkv) * D + c * CPL;
-  const size_t vstride = static_cast<size_t>(p.Hkv) * D;
-  for (int kb = t0; kb < t1; ++kb) {
-    int* kf = sKeep[kb & 1];
-    if (tid < GP) kf[tid] = tid < p.G ? p.keep[(r0 + tid) * p.nk + kb] : 0;
-    __syncthreads();  // also: the previous tile's sP has been read
-    int any = 0;
-#pragma unroll
-    for (int g = 0; g < GP; ++g) any |= kf[g];
-    if (!any) continue;  // uniform: V of this tile is not read
-    // V rows of my steps and the tile's P, loads issued together
-    uint32_t raw[KPW / 2][CPL / 2];
-#pragma unroll
-    for (int u = 0; u < KPW / 2; ++u) {
-      const int j = kb * BK + warp * KPW + u * 2 + half;
-      if (j < p.Lk) {
-        const uint16_t* src = vrow0 + static_cast<size_t>(j) * vstride;
-        if constexpr (CPL == 8) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
-          raw[u][0] = v.x; raw[u][1] = v.y; raw[u][2] = v.z; raw[u][3] = v.w;
-        } else {
-          const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-          raw[u][0] = v.x; raw[u][1] = v.y;
+  const uint32_t ring = smem_u32(smem + Lay::OFF_RING);
+  int base = 0;    // listed tiles of earlier segments (ring position)
+  int issued = 0;  // warp 8, lane 0: V loads issued (an abort stops the issue)
+  for (int seg0 = t0; seg0 < t1; seg0 += LIST) {
+    const int seg1 = min(seg0 + LIST, t1);
+    if (warp == 8) {  // the segment's list of tiles some head keeps, in order
+      int n = 0;
+      for (int k0 = seg0; k0 < seg1; k0 += 32) {
+        const int kb = k0 + lane;
+        uint32_t bits = 0;
+        if (kb < seg1)
+          for (int g = 0; g < p.G; ++g) bits |= p.keep[(r0 + g) * p.nk + kb] ? (1u << g) : 0u;
+        const unsigned any = __ballot_sync(0xffffffffu, bits != 0u);
+        const int at = n + __popc(any & ((1u << lane) - 1u));
+        if (bits) {
+          sList[at] = kb;
+          sBits[at] = static_cast<uint8_t>(bits);
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < CPL / 2; ++e) raw[u][e] = 0u;
+        n += __popc(any);
       }
-    }
-    for (int i = tid; i < GP * BK; i += 256) {
-      const int g = i / BK, j = i % BK;
-      float pv = 0.f;
-      if (kf[g]) pv = ex2_approx(p.scores[(r0 + g) * p.Lkp + static_cast<size_t>(kb) * BK + j] - sM[g]);
-      sP[g][j] = pv;  // keys past Lk have s = -inf: 0
+      if (lane == 0) *sCount = n;
     }
     __syncthreads();
-#pragma unroll
-    for (int u = 0; u < KPW / 2; ++u) {
-      const int jj = warp * KPW + u * 2 + half;
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float pg = sP[g][jj];
-#pragma unroll
-        for (int e = 0; e < CPL / 2; ++e) {
-          acc[g][2 * e] = fmaf(pg, bf16lo_to_f32(raw[u][e]), acc[g][2 * e]);
-          acc[g][2 * e + 1] = fmaf(pg, bf16hi_to_f32(raw[u][e]), acc[g][2 * e + 1]);
+    const int n = *sCount;
+    if (warp == 8) {
+      if (lane == 0) {
+        for (int i = 0; i < n; ++i) {
+          const int ig = base + i, st = ig % NS;
+          if (ig >= NS && !mbar_wait(&empty[st], ((ig / NS) - 1) & 1, fs)) break;
+          mbar_arrive_expect_tx(&full[st], TB);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(&tm_v, &full[st], smem + Lay::OFF_RING + st * TB + h * (BK * 128), h * 64, hkv,
+                        sList[i] * BK, b);
+          issued = ig + 1;
         }
       }
+    } else {
+      float scn[NPT];  // the scores of tile i + 1, loaded while tile i is used
+      auto load_scores = [&](int i) {
+        const int kb = sList[i];
+#pragma unroll
+        for (int k = 0; k < NPT; ++k) {
+          const int idx = tid + k * 256, g = idx / BK, j = idx % BK;
+          scn[k] = (idx < GP * BK && ((sBits[i] >> g) & 1u))
+                       ? __ldg(p.scores + (r0 + g) * p.Lkp + static_cast<size_t>(kb) * BK + j)
+                       : -INFINITY;
+        }
+      };
+      if (n > 0) load_scores(0);
+      for (int i = 0; i < n; ++i) {
+        const int ig = base + i, st = ig % NS;
+        float* P = sP + (ig & 1) * GP * BK;
+#pragma unroll
+        for (int k = 0; k < NPT; ++k) {
+          const int idx = tid + k * 256;
+          if (idx < GP * BK) P[idx] = scn[k] == -INFINITY ? 0.f : ex2_approx(scn[k] - sM[idx / BK]);
+        }
+        if (i + 1 < n) load_scores(i + 1);
+        named_bar_sync(1, 256);  // P of this tile is in place (and the one two tiles back is read)
+        const bool ok = mbar_wait_warp(&full[st], (ig / NS) & 1, fs);
+        if (ok) {
+#pragma unroll
+          for (int u = 0; u < KPW / 2; ++u) {
+            const int jj = warp * KPW + u * 2 + half;
+            uint32_t raw[CPL / 2];
+            if constexpr (CPL == 8) {
+              ld_shared_v4(dx_row_chunk<BK>(ring + st * TB, jj, c), raw[0], raw[1], raw[2], raw[3]);
+            } else {
+              uint32_t a0, a1, a2, a3;
+              ld_shared_v4(dx_row_chunk<BK>(ring + st * TB, jj, c >> 1), a0, a1, a2, a3);
+              raw[0] = (c & 1) ? a2 : a0;
+              raw[1] = (c & 1) ? a3 : a1;
+            }
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+              const float pg = P[g * BK + jj];
+#pragma unroll
+              for (int e = 0; e < CPL / 2; ++e) {
+                acc[g][2 * e] = fmaf(pg, bf16lo_to_f32(raw[e]), acc[g][2 * e]);
+                acc[g][2 * e + 1] = fmaf(pg, bf16hi_to_f32(raw[e]), acc[g][2 * e + 1]);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);  // my rows of this V stage are read
+      }
     }
+    base += n;
+    __syncthreads();  // the next segment's list overwrites this one
+  }
+  if (warp == 8) {  // the last loads have landed before the CTA ends
+    if (lane == 0)
+      for (int ig = max(0, issued - NS); ig < issued; ++ig) mbar_wait_drain(&full[ig % NS], (ig / NS) & 1);
+    return;
   }
   // sum the two halves, then the 8 warps
 #pragma unroll
   for (int g = 0; g < GP; ++g)
 #pragma unroll
     for (int e = 0; e < CPL; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], 16);
-  __syncthreads();
   if (half == 0)
 #pragma unroll
     for (int g = 0; g < GP; ++g)
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) sO[warp][g][c * CPL + e] = acc[g][e];
-  __syncthreads();
+      for (int e = 0; e < CPL; ++e) sO[(warp * GP + g) * (D + 4) + c * CPL + e] = acc[g][e];
+  named_bar_sync(1, 256);
   for (int i = tid; i < GP * D; i += 256) {
     const int g = i / D, col = i % D;
     if (g >= p.G) continue;
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) o += sO[w][g][col];
+    for (int w = 0; w < 8; ++w) o += sO[(w * GP + g) * (D + 4) + col];
     const float l = sLn[g];
     const size_t part = (r0 + g) * p.n_splits + sp;
     p.o_part[part * D + col] = l > 0.f ? o / l : 0.f;
