@@ -768,8 +768,9 @@ def run_reference(args):
 
 def run_kernel_case(args):
     """One op on a small case (inputs still larger than L2), for ncu captures:
-    fwd / bwd: B=1, Hq=Hkv=16, L=16384, d=128, tau=1; decode: B=8, Lk=32768,
-    Hq=32, Hkv=8, d=128. Runs warmup + steps calls and prints the mean ms."""
+    fwd / bwd: B=1, Hq=Hkv=16, L=16384, d=128, tau=1; decode and decode_exact:
+    B=8, Lk=32768, Hq=32, Hkv=8, d=128. Runs warmup + steps calls and prints the
+    mean ms."""
     import torch
     import mass_gated_causal_b200 as mala
     from workloads import TrainWorkload, DecodeWorkload, make_decode_inputs, make_train_inputs
@@ -797,8 +798,12 @@ def run_kernel_case(args):
         inp = make_decode_inputs(w, workers=default_workers())
         q, kc, vc = (to_dev(inp[x]) for x in ("q", "kcache", "vcache"))
 
-        def fn():
-            mala.decode(q, kc, vc, w.scale, 1.0, w.Bk)
+        if args.kernel == "decode":
+            def fn():
+                mala.decode(q, kc, vc, w.scale, 1.0, w.Bk)
+        else:
+            def fn():
+                mala.decode_exact(q, kc, vc, w.scale, 1.0, w.Bk)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -859,7 +864,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-blocks", type=int, default=16)
-    ap.add_argument("--kernel", choices=("fwd", "bwd", "decode"), default=None,
+    ap.add_argument("--kernel", choices=("fwd", "bwd", "decode", "decode_exact"), default=None,
                     help="run one op on a small case (for profiler captures) instead of the benchmark")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture (reported as is)")
