@@ -12,8 +12,9 @@ sub-objects of the same line.
              tiles (fwd 2d*N_legal + 2d*N_f, bwd 2d*N_legal + 8d*N_b), summed
              over ranks, divided by the max-over-ranks device time
   e2e        the same metric through the C ABI starting from pinned host
-             buffers: H2D of q, k, v, dO and D2H of dq, dk, dv inside the
-             timed region
+             buffers: every step's H2D of q, k, v, dO and D2H of dq, dk, dv
+             inside the timed region, overlapped with the neighbouring steps'
+             compute (two device buffer sets, a copy stream per direction)
   roofline   the dominant kernel's achieved rate against the measured peak
 
 Multi-GPU (torchrun): every rank runs its own copy of the workload (a per-GPU
@@ -313,18 +314,65 @@ def run_cuda(args):
     h2d = sum(t.numel() * 2 for t in (hq_, hk_, hv_, hdo_))
     d2h = sum(t.numel() * 2 for t in (hdq, hdk, hdv))
 
-    def e2e_fn(mid=None):
-        q.copy_(hq_, non_blocking=True)
-        k.copy_(hk_, non_blocking=True)
-        v.copy_(hv_, non_blocking=True)
-        do.copy_(hdo_, non_blocking=True)
-        train_step(tau)(mid)
-        hdq.copy_(dq, non_blocking=True)
-        hdk.copy_(dk, non_blocking=True)
-        hdv.copy_(dv, non_blocking=True)
+    # Each step copies its inputs in and reads its gradients back. Two device
+    # buffer sets and one stream per copy direction let the copies of steps
+    # n + 1 (in) and n (out) overlap the compute of step n, as a training loop
+    # with prefetching would; the timed region spans all K steps' copies and
+    # ends once the last gradients are on the host.
+    cp_in, cp_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    sets = [(q, k, v, do, dq, dk, dv), tuple(torch.empty_like(t) for t in (q, k, v, do, dq, dk, dv))]
+    ev_in = [torch.cuda.Event() for _ in range(2)]   # inputs of set s have landed
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]  # the step on set s is done
+    ev_out = [torch.cuda.Event() for _ in range(2)]  # gradients of set s are on the host
 
-    tote, _, _ = timed(e2e_fn, max(2, args.steps // 2), 1)
-    ms_e2e = max_over_ranks(float(np.mean(tote)))
+    def copy_in(s_):
+        with torch.cuda.stream(cp_in):
+            cp_in.wait_event(ev_cmp[s_])  # the step that last read set s_ is done
+            for dst, src in zip(sets[s_][:4], (hq_, hk_, hv_, hdo_)):
+                dst.copy_(src, non_blocking=True)
+            ev_in[s_].record(cp_in)
+
+    def step_on(s_, tau_):
+        q_, k_, v_, do_, dq_, dk_, dv_ = sets[s_]
+        stream.wait_event(ev_in[s_])
+        stream.wait_event(ev_out[s_])  # its gradient buffers were read back two steps ago
+        rc = mala.mala_fwd(q_, k_, v_, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, fws, fws_bytes, kept_f,
+                           None, stream)
+        assert rc == 0
+        rc = mala.mala_bwd(q_, k_, v_, o, do_, lse, dq_, dk_, dv_, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, ws,
+                           ws_bytes, kept_b, None, stream)
+        assert rc == 0
+        ev_cmp[s_].record(stream)
+        with torch.cuda.stream(cp_out):
+            cp_out.wait_event(ev_cmp[s_])
+            for dst, src in zip((hdq, hdk, hdv), (dq_, dk_, dv_)):
+                dst.copy_(src, non_blocking=True)
+            ev_out[s_].record(cp_out)
+
+    def e2e_run(nsteps):
+        copy_in(0)
+        for n_ in range(nsteps):
+            if n_ + 1 < nsteps:
+                copy_in((n_ + 1) & 1)
+            step_on(n_ & 1, tau)
+        stream.wait_event(ev_out[(nsteps - 1) & 1])
+
+    n_e2e = max(3, args.steps // 2)
+    e2e_run(max(3, args.warmup))
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    cp_in.wait_event(e_start)  # the first input copy is inside the timed region
+    e2e_run(n_e2e)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    assert mala.mala_check_status(stream) == 0
+    ms_e2e = max_over_ranks(e_start.elapsed_time(e_end) / n_e2e)
+    del sets
 
     # the same fwd+bwd step on the 128K workload (the metric is quoted at 32K and 128K)
     long_leg = None
@@ -382,7 +430,8 @@ def run_cuda(args):
                           "frac_of_peak": round(flops0 / (ms0 * 1e-3) / 1e12 / peak_t, 4),
                           "mala_speedup": round(ms0 / ms, 3)},
         "e2e": {"value": round(world * step_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "copies": "overlapped with compute (two buffer sets, a stream per direction)"},
         "roofline": roof,
         "gpu_launches": 5 * args.steps,
         "clocks": clocks,
