@@ -80,3 +80,10 @@ def test_decode_exact_fullsize_sampled(cuda_lib):
     rows = sorted({(0, 0), (C4.B - 1, C4.Hq - 1)} | {(int(rng.integers(C4.B)), int(rng.integers(C4.Hq)))
                                                        for _ in range(10)})
     run_case(cuda_lib, C4, 1.0, split_counts=(0, 1), rows=rows, workers=default_workers())
+
+
+def test_decode_exact_long_split_segments(cuda_lib):
+    """A split of more than 1024 tiles (one split over 70000 keys in 64-key
+    tiles) is listed and streamed in segments; two splits take one each."""
+    w = DecodeWorkload("exact_long", 1, 4, 2, 70000, 64, 64, seed=8101)
+    run_case(cuda_lib, w, 1.0, split_counts=(1, 2))
