@@ -13,7 +13,10 @@
 // query block when Bq = 128 and two when Bq = 64; decisions are per block.
 // The same kernel runs prefill against an existing cache: query row r sits at
 // position P0 + r (P0 = Lk - Lq), sees keys 0 .. P0 + r and uses Lq = P0 + r + 1
-// in its threshold; the training forward is P0 = 0, Lq = Lk.
+// in its threshold; the training forward is P0 = 0, Lq = Lk. In a packed batch
+// (device cu_seqlens) each CTA takes its sequence's lengths and row offsets
+// from the tables, and a partial last tile of O is stored row by row so that
+// the next sequence's rows are not written.
 //   warps 0-3  softmax warpgroup of tile A (thread t = row t = TMEM lane t)
 //   warps 4-7  softmax warpgroup of tile B
 //   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring,
