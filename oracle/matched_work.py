@@ -15,9 +15,9 @@ This module does that on synthetic inputs. For every query row i:
 - omitted mass 1 - sum of the retained p_ij, and the relative L2 error of each
   output against the dense output.
 
-``matched_work`` returns per-row arrays and ``summary`` aggregates them; run
-``python -m oracle.matched_work`` for a report on the 1K and 8K workloads.
-Only tests and analysis scripts import this module.
+``matched_work`` returns per-row arrays and ``summary`` aggregates them;
+``tests/report_matched_work.py`` prints the report on the 1K and 8K workloads.
+Only tests import this module.
 """
 from __future__ import annotations
 
@@ -95,23 +95,3 @@ def summary(r) -> dict:
         "err_ref_mean": float(r["err_ref"].mean()),
         "rows_within_10pct": float(np.mean(r["omit_mala"] <= 1.1 * r["omit_ref"] + 1e-15)),
     }
-
-
-def _report():
-    import math
-    import sys
-    import os
-    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
-    from workloads import C0, C1, bf16_bits_to_f64, make_train_inputs
-    cases = [(C0, None), (C1, [(0, h) for h in range(4)])]
-    for w, heads in cases:
-        t = make_train_inputs(w)
-        q, k, v = (bf16_bits_to_f64(t[x]) for x in ("q", "k", "v"))
-        for tau in (0.5, 1.0, 4.0, 16.0):
-            s = summary(matched_work(q, k, v, 1 / math.sqrt(w.d), tau, w.Bq, w.Bk, heads=heads))
-            print(w.name, "heads", "all" if heads is None else len(heads), "tau", tau,
-                  {x: (round(y, 6) if isinstance(y, float) else y) for x, y in s.items()}, flush=True)
-
-
-if __name__ == "__main__":
-    _report()
