@@ -69,6 +69,27 @@ def train_flops(d: int, B: int, Hq: int, L: int, live: np.ndarray, keep_f, keep_
             "fwd": 2 * d * n_legal + 2 * d * n_f, "bwd": 2 * d * n_legal + 8 * d * n_b}
 
 
+def packed_flops(lens, Hq, d, Bq, Bk, keep_f, keep_b):
+    """Effective FLOPs of one fwd and one bwd of a packed training batch: each
+    sequence's live pairs with its corner [nq_s, nk_s] of the keep maps
+    [S, Hq, max_nq, max_nk] (None = all kept). Also returns the legal-tile count
+    and the kept fwd / bwd tiles."""
+    fl = {"n_legal": 0, "n_f": 0, "n_b": 0, "fwd": 0, "bwd": 0, "tiles": 0, "kept_f": 0, "kept_b": 0}
+    for s_, L in enumerate(lens):
+        live = live_pairs(L, Bq, Bk)
+        a, b_ = live.shape
+        kf = None if keep_f is None else keep_f[s_:s_ + 1, :, :a, :b_]
+        kb = None if keep_b is None else keep_b[s_:s_ + 1, :, :a, :b_]
+        f1 = train_flops(d, 1, Hq, L, live, kf, kb)
+        for key_ in ("n_legal", "n_f", "n_b", "fwd", "bwd"):
+            fl[key_] += f1[key_]
+        n_t = Hq * int((live > 0).sum())
+        fl["tiles"] += n_t
+        fl["kept_f"] += n_t if kf is None else int((kf == 1).sum())
+        fl["kept_b"] += n_t if kb is None else int((kb == 1).sum())
+    return fl
+
+
 def decode_bytes(B, Hq, Hkv, Lk, d, Bk, keep_map):
     """Algorithmic bytes of one decode step: all K, V of tiles kept by >= 1 head of
     the group, q in and o out (bf16)."""
@@ -553,20 +574,9 @@ def run_varlen_leg(w, mala, torch, dev, stream, pk, workers, timed, max_over_ran
     assert mala.mala_check_status(stream) == 0
     kmf, kmb = km_f.cpu().numpy(), km_b.cpu().numpy()
     del km_f, km_b
-    fl = {"n_legal": 0, "n_f": 0, "n_b": 0, "fwd": 0, "bwd": 0}
-    fl0 = dict(fl)
-    n_tiles = kept_tf = kept_tb = 0
-    for s_, L in enumerate(w.lens):  # per sequence: its own live pairs and its corner of the keep maps
-        live = live_pairs(L, w.Bq, w.Bk)
-        a, b_ = live.shape
-        f1 = train_flops(d, 1, Hq, L, live, kmf[s_:s_ + 1, :, :a, :b_], kmb[s_:s_ + 1, :, :a, :b_])
-        f0 = train_flops(d, 1, Hq, L, live, None, None)
-        for key_ in fl:
-            fl[key_] += f1[key_]
-            fl0[key_] += f0[key_]
-        n_tiles += Hq * int((live > 0).sum())
-        kept_tf += int((kmf[s_, :, :a, :b_] == 1).sum())
-        kept_tb += int((kmb[s_, :, :a, :b_] == 1).sum())
+    fl = packed_flops(w.lens, Hq, d, w.Bq, w.Bk, kmf, kmb)
+    fl0 = packed_flops(w.lens, Hq, d, w.Bq, w.Bk, None, None)
+    n_tiles, kept_tf, kept_tb = fl["tiles"], fl["kept_f"], fl["kept_b"]
     out = {"workload": w.name, "lens": list(w.lens), "total": T, "Hq": Hq, "Hkv": Hkv, "d": d, "Bq": w.Bq,
            "Bk": w.Bk, "steps": steps, "warmup": warmup,
            "retained_tiles": {"fwd": round(kept_tf / n_tiles, 4), "bwd": round(kept_tb / n_tiles, 4),

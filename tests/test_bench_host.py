@@ -65,3 +65,26 @@ def test_profiled_traffic_tracks_kernel_sources(tmp_path, monkeypatch):
     assert bench.profiled_traffic("mala_bwd_kernel", "w") == 1234.5
     (csrc / "mala_bwd.cuh").write_text("kernel v2\n")  # the kernel changed since the capture
     assert bench.profiled_traffic("mala_bwd_kernel", "w") is None
+
+
+def test_packed_flops_sum_per_sequence():
+    """Packed accounting: at tau = 0 every sequence contributes its causal
+    triangle (L(L+1)/2 live pairs per head); with keep maps, exactly the live
+    pairs of the kept tiles of each sequence's corner count."""
+    lens, Hq, d, Bt = [5, 17, 0, 9], 2, 8, 4
+    fl0 = bench.packed_flops(lens, Hq, d, Bt, Bt, None, None)
+    tri = sum(L * (L + 1) // 2 for L in lens) * Hq
+    assert fl0["n_legal"] == fl0["n_f"] == fl0["n_b"] == tri
+    assert fl0["fwd"] == 4 * d * tri and fl0["bwd"] == 10 * d * tri
+    assert fl0["tiles"] == fl0["kept_f"] == Hq * sum(n * (n + 1) // 2 for n in (2, 5, 0, 3))
+    rng = np.random.default_rng(0)
+    km = rng.integers(0, 2, size=(4, Hq, 5, 5)).astype(np.uint8)
+    fl = bench.packed_flops(lens, Hq, d, Bt, Bt, km, km)
+    want = 0
+    for s, L in enumerate(lens):  # live pairs (i, j <= i) of kept tiles, counted one by one
+        for h in range(Hq):
+            for i in range(L):
+                for j in range(i + 1):
+                    want += int(km[s, h, i // Bt, j // Bt] == 1)
+    assert fl["n_f"] == fl["n_b"] == want
+    assert fl["fwd"] == 2 * d * tri + 2 * d * want and fl["bwd"] == 2 * d * tri + 8 * d * want
