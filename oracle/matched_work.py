@@ -30,16 +30,24 @@ def _rows_of_block(L, Bq, qb):
     return np.arange(qb * Bq, min((qb + 1) * Bq, L))
 
 
-def matched_work(q, k, v, scale: float, tau: float, Bq: int, Bk: int, heads=None):
+def matched_work(q, k, v, scale: float, tau: float, Bq: int, Bk: int, heads=None, keep=None):
     """q [B,L,Hq,d], k/v [B,L,Hkv,d] fp64. Returns a dict of per-row arrays over
     the selected (b, hq) (default all): slots, live, omit_mala, omit_ref,
-    err_mala, err_ref (relative L2 error of the row's output)."""
+    err_mala, err_ref (relative L2 error of the row's output).
+
+    With ``keep`` (a keep map [B,Hq,nq,nk] from elsewhere, e.g. the CUDA
+    forward's) the retained keys come from that map and MALA's output is the
+    softmax over them -- what the forward computes with those decisions, up to
+    rounding; without it, the oracle forward decides and supplies its output."""
     q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
-    f = _mala_fwd(q, k, v, scale, tau, Bq, Bk)
-    keep, o_mala = f["keep"], f["o"]
+    if keep is None:
+        f = _mala_fwd(q, k, v, scale, tau, Bq, Bk)
+        keep, o_mala = f["keep"], f["o"]
+    else:
+        o_mala = None
     nq = -(-L // Bq)
     if heads is None:
         heads = [(b, h) for b in range(B) for h in range(Hq)]
@@ -77,7 +85,12 @@ def matched_work(q, k, v, scale: float, tau: float, Bq: int, Bk: int, heads=None
             out["live"].append(live.sum(axis=1))
             out["omit_mala"].append(omit_mala)
             out["omit_ref"].append(omit_ref)
-            out["err_mala"].append(np.linalg.norm(o_mala[b, rows, h] - o_dense, axis=1) / nrm)
+            if o_mala is None:  # the softmax over MALA's retained keys
+                pm = p * ret
+                om = (pm @ vv) / pm.sum(axis=1, keepdims=True)
+            else:
+                om = o_mala[b, rows, h]
+            out["err_mala"].append(np.linalg.norm(om - o_dense, axis=1) / nrm)
             out["err_ref"].append(np.linalg.norm(o_ref - o_dense, axis=1) / nrm)
     return {x: np.concatenate(v_) for x, v_ in out.items()}
 

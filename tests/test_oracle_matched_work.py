@@ -76,3 +76,21 @@ def test_tau0_retains_everything():
     assert (r["slots"] == r["live"]).all()
     assert np.abs(r["omit_mala"]).max() < 1e-12 and np.abs(r["omit_ref"]).max() < 1e-12
     assert r["err_mala"].max() < 1e-12 and r["err_ref"].max() < 1e-12
+
+
+def test_given_keep_map_equals_the_oracle_decisions():
+    # the analysis of a keep map passed in (as the CUDA forward's is) equals the
+    # analysis of the oracle's own decisions when the maps are the same
+    q, k, v, _ = case(200, 16, 2, 1, seed=162, sharpen=2.0)
+    from oracle import fwd
+    keep = fwd(q, k, v, 0.25, 1.0, 16, 16)["keep"]
+    a = matched_work(q, k, v, 0.25, 1.0, 16, 16)
+    b = matched_work(q, k, v, 0.25, 1.0, 16, 16, keep=keep)
+    for name in a:
+        assert np.abs(a[name] - b[name]).max() < 1e-12, name
+    # a different map changes the slots and the masses accordingly
+    keep2 = keep.copy()
+    keep2[0, 0, 5, 2] = 1 - keep2[0, 0, 5, 2]
+    c = matched_work(q, k, v, 0.25, 1.0, 16, 16, keep=keep2)
+    rows = slice(5 * 16, 6 * 16)
+    assert (np.abs(c["slots"][rows] - a["slots"][rows]) == 16).all()
