@@ -79,11 +79,8 @@ MALA_API int mala_abi_version(void);
  * row r with a live key satisfies
  *     max_live_j exp(s_rj - m_r) / l_r >= tau / (i_r + 1)      (ties keep).
  * A kept tile updates (m, l) and O for every row of the block; a skipped
- * tile does no softmax update and no PV. V tiles are fetched ahead for every
- * tile, kept or not (they come from L2 and the kernel is not memory-bound;
- * fetching only after the vote measured slower), so a skip saves the softmax
- * update and the PV but not the V load; mala_decode keeps the strict rule.
- * The PV product runs in
+ * tile does no V load, no softmax update and no PV: with tau > 0 the V tile
+ * is requested only after a query block's vote has kept it. The PV product runs in
  * fp16 on an fp16 copy of V made by the call in `workspace`; V values must lie
  * inside the fp16 range (|v| <= 65504); larger ones are clamped and reported
  * as MALA_ERR_RANGE by mala_check_status.
@@ -356,14 +353,39 @@ MALA_API int mala_decode_paged(const void* q, const void* k_pages, const void* v
  * workspace. A problem whose partials need more than the fixed array
  * (mala_decode_workspace_size(B, Hq, d, n_splits used) > 8 MiB) returns
  * MALA_ERR_WORKSPACE and launches nothing. The first call on a device looks
- * up the array's device address for that device (so make that first call
- * before any stream capture). All calls share the array: calls that overlap
- * on the GPU race and must be serialised by the caller.
+ * up the array's device address for that device and caches it with the id of
+ * the CUDA context current at the time; a call that finds another context
+ * current (after cudaDeviceReset, for instance) looks it up again. Make the
+ * first call, and the first after such a reset, before any stream capture.
+ * All calls share the array: calls that overlap on the GPU race and must be
+ * serialised by the caller.
  */
 MALA_API size_t mala_decode_noalloc_max_bytes(void);
 MALA_API int mala_decode_noalloc(const void* q, const void* kcache, const void* vcache, void* o, float* lse,
                                  int B, int Hq, int Hkv, int Lk, int d, float scale, float tau, int Bk,
                                  int n_splits, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
+
+/*
+ * mala_test_hooks -- switches for tests of the failure path and of the V
+ * traffic. Process-wide; they apply to calls enqueued after this one (on any
+ * stream) until changed, and are not meant for production use. The pages
+ * describe nothing of the kind.
+ *
+ *   wait_limit_ns  limit of each bounded device-side wait; 0 restores the
+ *                  default (2 s)
+ *   stall_tile     -1: off. >= 0: the MMA issuer of mala_fwd / mala_prefill /
+ *                  mala_fwd_varlen / mala_bwd / mala_bwd_varlen, and the K
+ *                  producer of mala_decode / mala_decode_paged /
+ *                  mala_decode_noalloc, wait before key tile `stall_tile` on a
+ *                  barrier nothing completes, so that the wait expires: the
+ *                  kernel then leaves through its abort path and
+ *                  mala_check_status returns MALA_ERR_DEVICE_TIMEOUT. Outputs
+ *                  of such a call are undefined.
+ *   fwd_v_tiles    NULL: off. Else a DEVICE uint64 the forward kernels (gate
+ *                  on) increase by one for every V tile they load.
+ * Returns MALA_ERR_INVALID_ARG for stall_tile < -1, else MALA_OK.
+ */
+MALA_API int mala_test_hooks(unsigned long long wait_limit_ns, int stall_tile, unsigned long long* fwd_v_tiles);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's status

@@ -39,7 +39,7 @@ EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_prefill"
             "mala_fwd_workspace_size", "mala_bwd_workspace_size", "mala_bwd", "mala_bwd_varlen",
             "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_paged",
             "mala_decode_exact_workspace_size", "mala_decode_exact",
-            "mala_decode_noalloc_max_bytes", "mala_decode_noalloc", "mala_check_status")
+            "mala_decode_noalloc_max_bytes", "mala_decode_noalloc", "mala_test_hooks", "mala_check_status")
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _lib.mala_status_string.argtypes = [_i]
@@ -81,6 +81,8 @@ _lib.mala_decode.restype = _i
 _lib.mala_decode_noalloc_max_bytes.restype = _sz
 _lib.mala_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _vp, _vp]
 _lib.mala_decode_noalloc.restype = _i
+_lib.mala_test_hooks.argtypes = [ctypes.c_ulonglong, _i, _vp]
+_lib.mala_test_hooks.restype = _i
 _lib.mala_check_status.argtypes = [_vp]
 _lib.mala_check_status.restype = _i
 
@@ -213,6 +215,10 @@ def mala_decode_noalloc(q, kcache, vcache, o, lse, B, Hq, Hkv, Lk, d, scale, tau
     return int(_lib.mala_decode_noalloc(_p(q), _p(kcache), _p(vcache), _p(o), _p(lse), B, Hq, Hkv, Lk, d,
                                         float(scale), float(tau), Bk, n_splits, _p(kept_tiles), _p(keep_map),
                                         _stream(stream)))
+
+
+def mala_test_hooks(wait_limit_ns: int = 0, stall_tile: int = -1, fwd_v_tiles=None) -> int:
+    return int(_lib.mala_test_hooks(int(wait_limit_ns), int(stall_tile), _p(fwd_v_tiles)))
 
 
 def mala_check_status(stream=None) -> int:

@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -23,6 +24,11 @@
 namespace {
 
 __device__ unsigned int g_mala_status;  // per-device status word, see mala_check_status
+
+// Test hooks (mala_test_hooks): bounded-wait limit, stall tile, V-tile counter.
+std::atomic<unsigned long long> g_wait_ns{mala::kWaitLimitNs};
+std::atomic<int> g_stall_tile{-1};
+std::atomic<unsigned long long*> g_v_tiles{nullptr};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -133,7 +139,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned n_chunks = (p.n_pairs + p.chunk_pairs - 1) / p.chunk_pairs;
   const unsigned grid = n_chunks * p.chunk_pairs * p.B * p.Hq;
-  kern<<<grid, 320, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mo, p);
+  kern<<<grid, 352, Lay::ALLOC_BYTES, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
@@ -311,6 +317,9 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   p.kept_tiles = kept_tiles;
   p.keep_map = keep_map;
   p.status = status;
+  p.v_tiles = g_v_tiles.load();
+  p.wait_ns = g_wait_ns.load();
+  p.stall_tile = g_stall_tile.load();
   if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
   const long long n8 = static_cast<long long>(tb) * tk * Hkv * d / 8;
   const int cv_grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148LL * 16));
@@ -415,6 +424,8 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const vo
   p.kept_tiles = kept_tiles;
   p.keep_map = keep_map;
   p.status = status;
+  p.wait_ns = g_wait_ns.load();
+  p.stall_tile = g_stall_tile.load();
 
   const long long chunks = static_cast<long long>(tb) * tl * Hq * (d / 8);  // 16-byte chunks of O / dO
   const int pre_grid = static_cast<int>(std::min<long long>((chunks + 255) / 256, 148LL * 16));
@@ -552,6 +563,8 @@ int run_decode(const void* q, const CUtensorMap& mk, const CUtensorMap& mv, void
   p.kept_tiles = kept_tiles;
   p.keep_map = keep_map;
   p.status = status;
+  p.wait_ns = g_wait_ns.load();
+  p.stall_tile = g_stall_tile.load();
   if (cudaMemsetAsync(kept_tiles, 0, sizeof(int32_t) * B * Hq, st) != cudaSuccess) return MALA_ERR_CUDA;
   const bool gate = tau > 0.f;
   int rc;
@@ -678,6 +691,7 @@ int mala_decode_exact(const void* q, const void* kcache, const void* vcache, voi
   unsigned* status = status_ptr();
   if (!status) return MALA_ERR_CUDA;
   p.status = status;
+  p.wait_ns = g_wait_ns.load();
   CUtensorMap mv;
   if (!make_bshd_map(&mv, vcache, B, Lk, Hkv, d, Bk)) return MALA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -685,6 +699,14 @@ int mala_decode_exact(const void* q, const void* kcache, const void* vcache, voi
   if (d == 64 && Bk == 128) return launch_dx_g<64, 128>(mv, p, st);
   if (d == 128 && Bk == 64) return launch_dx_g<128, 64>(mv, p, st);
   return launch_dx_g<64, 64>(mv, p, st);
+}
+
+int mala_test_hooks(unsigned long long wait_limit_ns, int stall_tile, unsigned long long* fwd_v_tiles) {
+  if (stall_tile < -1) return MALA_ERR_INVALID_ARG;
+  g_wait_ns.store(wait_limit_ns == 0 ? mala::kWaitLimitNs : wait_limit_ns);
+  g_stall_tile.store(stall_tile);
+  g_v_tiles.store(fwd_v_tiles);
+  return MALA_OK;
 }
 
 int mala_check_status(void* stream) {
@@ -716,8 +738,12 @@ int mala_check_status(void* stream) {
 //
 // The array's name is only a host-side stand-in in host code; its device
 // address is looked up with cudaGetSymbolAddress the first time the entry
-// point runs on a device (with that device current) and cached per device.
-// That first call should therefore come before any stream capture.
+// point runs on a device (with that device current) and cached per device,
+// together with the unique id of the CUDA context it was looked up in. A
+// call that finds another context current (after cudaDeviceReset, say, the
+// library's module lives in a new primary context) looks the address up
+// again. The first call on a device, and the first after such a reset, should
+// therefore come before any stream capture.
 //
 // All calls share the array and it keeps the last call's contents. Every
 // call overwrites all of the split partials it reads (empty splits included),
@@ -731,19 +757,53 @@ __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;  // 0: nothing cached
+  void* ptr = nullptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
 
-// Device address of g_decode_scratch on the current device (set-up on first use).
+// Unique id of the current CUDA context (driver entry points fetched at run
+// time, as for the tensor maps); false if there is none or the driver lacks
+// the calls.
+bool current_context_id(unsigned long long* id) {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+    return false;
+  return get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
+
+// Device address of g_decode_scratch on the current device (set-up on first
+// use in each context).
 void* decode_scratch_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    g_scratch_ptr[dev] = p;
-  }
-  return g_scratch_ptr[dev];
+  unsigned long long id = 0;
+  ScratchAddr& e = g_scratch_addr[dev];
+  if (e.ptr != nullptr && current_context_id(&id) && id == e.ctx_id) return e.ptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
+  // the look-up has made the device's context current if it was not; without
+  // a context id the address is not cached and is looked up on every call
+  e.ctx_id = current_context_id(&id) ? id : 0;
+  e.ptr = e.ctx_id != 0 ? p : nullptr;
+  return p;
 }
 
 }  // namespace

@@ -55,6 +55,8 @@ struct BwdParams {
   int32_t* kept_tiles;
   uint8_t* keep_map;
   unsigned* status;
+  uint64_t wait_ns;  // limit of each bounded wait
+  int stall_tile;    // test hook (-1: off): the MMA thread stalls before this tile
 };
 
 constexpr uint32_t kBwdAny = 1u << 4;
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(448, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
-  const FailState fs{abort_flag, p.status};
+  const FailState fs{abort_flag, p.status, p.wait_ns};
   // TMEM: two 128-column regions taken by tiles in turn (tile t uses region
   // t & 1 for S, then dP, then dQ), then dK and dV.
   const uint32_t tDK = tmem + 256, tDV = tmem + 256 + D;
@@ -281,6 +283,9 @@ __global__ void __launch_bounds__(448, 1)
         const int hq = walk_hq(t);
         const int i0 = walk_qs(t) * 128;
         const uint32_t tR = tmem + (t & 1) * 128;
+        // test hook: wait on a barrier only this thread completes (after the
+        // loop), so the bounded wait expires and the CTA takes its abort path
+        if (t == p.stall_tile && !mbar_wait(mma_final, 0, fs)) break;
         // the gate's decision (the compute warps have read S(t) out of the
         // region before voting) and dO(t), loaded ahead: one wait for both
         if (!mbar_wait2(dec_bar, t & 1, do_full, t & 1, fs)) break;

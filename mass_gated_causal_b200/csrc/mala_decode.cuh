@@ -52,6 +52,8 @@ struct DecParams {
   int32_t* kept_tiles;
   uint8_t* keep_map;  // [B, Hq, nk], nullable
   unsigned* status;
+  uint64_t wait_ns;  // limit of each bounded wait
+  int stall_tile;    // test hook (-1: off): the K producer stalls before this tile
 };
 
 // Sum N per-lane values over the L lanes of a group (lane index c = lane % L,
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(320, 1)
   const int t0 = bad ? nk : min(sp_idx * tps, nk);
   const int t1 = bad ? nk : min(t0 + tps, nk);
   const int T = t1 - t0;  // tiles kb = t1-1 ... t0
-  const FailState fs{abort_flag, p.status};
+  const FailState fs{abort_flag, p.status, p.wait_ns};
   // paged cache: the page of key tile kb, checked (an id outside the pool is
   // reported and read as zeros: a TMA load outside the tensor fills)
   auto page_of = [&](int kb) {
@@ -217,6 +219,9 @@ __global__ void __launch_bounds__(320, 1)
         const int pg = pg_next;
         if (kPaged && t + 1 < T) pg_next = page_of(t1 - 2 - t);
         if (t >= NK && !mbar_wait(&k_empty[st], ((t / NK) - 1) & 1, fs)) break;
+        // test hook: the phase that completes once tile t itself has been
+        // consumed never completes before tile t is loaded, so the wait expires
+        if (t == p.stall_tile && !mbar_wait(&k_empty[st], (t / NK) & 1, fs)) break;
         const int krow = kPaged ? 0 : (t1 - 1 - t) * BK, kouter = kPaged ? pg : b;
         if (kPaged) sPage[t & 7] = pg;  // for the gate warp's V request (it trails by < 8 tiles)
         mbar_arrive_expect_tx(&k_full[st], TB);

@@ -52,6 +52,7 @@ struct DxParams {
   void* o_out;          // [B, Hq, d] bf16 (written by the merge)
   float* lse_out;       // [B, Hq]
   unsigned* status;
+  uint64_t wait_ns;     // limit of each bounded wait
 };
 
 // Shared-memory layout of the PV kernel: an NS-stage ring of
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(288, 1) mala_dx_pv_kernel(const __grid_constan
     }
   }
   __syncthreads();
-  const FailState fs{abort_flag, p.status};
+  const FailState fs{abort_flag, p.status, p.wait_ns};
   const int c = lane & 15, half = lane >> 4;
   float acc[GP][CPL];
 #pragma unroll

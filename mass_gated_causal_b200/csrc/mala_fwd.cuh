@@ -19,24 +19,26 @@
 // the next sequence's rows are not written.
 //   warps 0-3  softmax warpgroup of tile A (thread t = row t = TMEM lane t)
 //   warps 4-7  softmax warpgroup of tile B
-//   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring,
-//              V tiles (fetched or passed over) through an NV ring
+//   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring
+//              (and, with the gate off, every V tile through the NV ring)
 //   warp  9    MMA issuer (one thread)
+//   warp  10   V issuer (one thread, gate on)
 // TMEM: S_A | S_B | O_A | O_B. P (fp16) is written over the first half of its
 // tile's S columns and read from TMEM by the PV MMA (A operand in TMEM).
 // The MMA thread alternates between the tiles -- PV_A(t), QK_A(t+1), PV_B(t),
 // QK_B(t+1) -- so the tensor core works on one tile while the other tile's
 // warpgroup runs its gate and softmax.
 //
-// V is fetched ahead for every tile, kept or not; a skipped tile gets no
-// softmax update and no PV, and its V tile is never read. The pages list V
-// loads among the work a skip saves; here they are kept on purpose. A CTA's K
-// and V tiles come from L2 (the CTAs of one KV head run together), the kernel
-// is bound by the softmax and the QK -> softmax -> PV chain rather than by
-// memory, and a V load requested only after the vote put its latency on that
-// chain: measured at 32K, GQA 32/8, fetching every V was faster at tau = 1, 4
-// and 16 than fetching V only for kept tiles (or for predicted ones). The
-// memory-bound decode kernel keeps the strict rule.
+// With the gate on, a V tile is requested only once a query block has voted
+// to keep it, so a skipped tile costs no V traffic. Both warpgroups vote on
+// every key tile t and post their votes to a mailbox in shared memory (a flag
+// ring and a sequence number per warpgroup). The V issuer reads tile A's vote
+// on t as soon as it is posted and, if A keeps t, requests V(t) at once, so
+// the load overlaps A's probability pass; otherwise it waits for B's vote. If
+// neither keeps t, nothing is loaded. V tiles take the NV slots in load order
+// (the n-th loaded tile uses slot n % NV); the MMA thread, which sees both
+// decisions of every tile, counts the loads the same way, and no barrier phase
+// stands for a tile that was not loaded.
 //
 // Precision: S = Q K^T is bf16 x bf16 -> fp32. PV runs in fp16 x fp16 -> fp32:
 // P is at most 2^8 (lazy-rescale bound) and V is read from an fp16 copy made
@@ -63,8 +65,12 @@ struct FwdParams {
   int32_t* kept_tiles;
   uint8_t* keep_map;
   unsigned* status;
+  unsigned long long* v_tiles;  // nullable test counter: V tiles loaded (one per load)
+  uint64_t wait_ns;             // limit of each bounded wait
+  int stall_tile;               // test hook (-1: off): the MMA thread stalls before this tile
 };
 
+constexpr int kVoteRing = 8;        // V mailbox depth (tiles a warpgroup may vote ahead of the V issuer)
 constexpr uint32_t kDecPV = 1u;     // some query block of the tile keeps it
 constexpr uint32_t kDecAbort = 2u;  // a wait gave up somewhere in the CTA
 constexpr unsigned kStatusRange = 2u;
@@ -84,7 +90,7 @@ struct FwdLayout {
   // sm_done[2], dec[2], pv_done[2], mma_final
   static constexpr int N_BARS = 1 + 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-  static constexpr int MISC_BYTES = 128;
+  static constexpr int MISC_BYTES = 192;
   static constexpr int BYTES = OFF_MISC + MISC_BYTES;
   static constexpr int ALLOC_BYTES = BYTES + 1024;  // slack for 1024-B alignment
   static constexpr int COL_S = 0;                   // S_A at 0, S_B at BK
@@ -106,7 +112,7 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 }
 
 template <int D, int BQ, int BK, bool kGate>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     mala_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
@@ -138,6 +144,8 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* dec_flags = misc + 2;  // [2] per tile
   uint32_t* vote = misc + 4;       // [2 tiles][2 parity][4 warps]
   uint32_t* evote = misc + 20;     // [2 tiles][4 warps]
+  uint32_t* vseq = misc + 28;      // [2] votes posted by each warpgroup (the V mailbox)
+  uint32_t* vflag = misc + 32;     // [2][kVoteRing] vote of tile t at t % kVoteRing: 1 keep, 2 abort
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -190,6 +198,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
+    vseq[0] = vseq[1] = 0u;
     fence_mbar_init();
   }
   if (warp == 8) {
@@ -206,7 +215,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
-  const FailState fs{abort_flag, p.status};
+  const FailState fs{abort_flag, p.status, p.wait_ns};
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -225,9 +234,7 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_4d(&tm_k, &k_full[st], sK + st * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, k_off + kb * BK,
                       bt);
         issued = t + 1;
-        // V(t) is fetched ahead into slot t % NV whatever the vote decides
-        // (see the note on V above)
-        {
+        if (!kGate) {  // no gate: every tile is kept (load t is tile t), so V(t) is fetched ahead into slot t % NV
           const int vs = t % NV;
           if (t >= NV && !mbar_wait(&v_empty[vs], ((t / NV) - 1) & 1, fs)) break;
           mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
@@ -239,7 +246,8 @@ __global__ void __launch_bounds__(320, 1)
       }
       mbar_wait_drain(bar_q, 0);
       for (int t = max(0, issued - NK); t < issued; ++t) mbar_wait_drain(&k_full[t % NK], (t / NK) & 1);
-      for (int t = max(0, vissued - NV); t < vissued; ++t) mbar_wait_drain(&v_full[t % NV], (t / NV) & 1);
+      if (!kGate)
+        for (int t = max(0, vissued - NV); t < vissued; ++t) mbar_wait_drain(&v_full[t % NV], (t / NV) & 1);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -277,8 +285,15 @@ __global__ void __launch_bounds__(320, 1)
         issue_qk(1, 0);
         umma_commit(&k_empty[0]);
       }
+      // V tiles occupy the slots in load order: the n-th loaded tile (a tile
+      // some query block of the pair keeps) uses slot n % NV
+      int nload = 0;
       for (int t = 0; ok && t < T; ++t) {
-        const int vslot = t % NV;
+        const int vslot = nload % NV;
+        // test hook: wait on a barrier only this thread completes (after the
+        // loop), so the bounded wait expires and the CTA takes its abort path
+        if (t == p.stall_tile && !mbar_wait(mma_final, 0, fs)) break;
+        bool v_waited = false;
         for (int x = 0; x < 2 && ok; ++x) {
           if (!mbar_wait(&dec_bar[x], t & 1, fs)) { ok = false; break; }
           const uint32_t dec = *reinterpret_cast<volatile uint32_t*>(&dec_flags[x]);
@@ -286,7 +301,8 @@ __global__ void __launch_bounds__(320, 1)
           const bool keep = (dec & kDecPV) != 0;
           if (!mbar_wait(&sm_done[x], t & 1, fs)) { ok = false; break; }  // P_x(t) written (or S_x released)
           if (keep) {
-            if (!mbar_wait(&v_full[vslot], (t / NV) & 1, fs)) { ok = false; break; }
+            if (!v_waited && !mbar_wait(&v_full[vslot], (nload / NV) & 1, fs)) { ok = false; break; }
+            v_waited = true;
             tc_fence_after();
             issue_pv(x, vslot);
           }
@@ -298,9 +314,60 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&v_empty[vslot]);  // V(t) read by both PVs (or not needed)
+        if (v_waited) {
+          umma_commit(&v_empty[vslot]);  // V(t) read by both PVs
+          ++nload;
+        }
       }
       umma_commit(mma_final);  // completes once every MMA above has finished
+    }
+    __syncwarp();
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ V issuer
+    if (kGate && lane == 0) {
+      // the vote of warpgroup x on tile t (bit 0 keep, bit 1 abort), once posted;
+      // a bounded wait like every other
+      auto vote_of = [&](int x, int t) -> uint32_t {
+        const volatile uint32_t* seq = reinterpret_cast<volatile uint32_t*>(vseq);
+        uint64_t t0 = 0;
+        for (uint32_t n = 0; seq[x] < static_cast<uint32_t>(t + 1); ++n) {
+          __nanosleep(32);
+          if ((n & 63u) == 63u) {
+            if (abort_raised(fs)) return 2u;
+            const uint64_t now = global_timer_ns();
+            if (t0 == 0) {
+              t0 = now;
+            } else if (now - t0 > fs.limit_ns) {
+              raise_abort(fs);
+              return 2u;
+            }
+          }
+        }
+        __threadfence_block();
+        return reinterpret_cast<volatile uint32_t*>(vflag)[x * kVoteRing + t % kVoteRing];
+      };
+      int n = 0;  // V tiles loaded so far; load n goes to slot n % NV
+      for (int t = 0; t < T; ++t) {
+        uint32_t f = vote_of(0, t);
+        if (f & 2u) break;
+        if (!(f & 1u)) {
+          f = vote_of(1, t);
+          if (f & 2u) break;
+        }
+        if (!(f & 1u)) continue;  // neither tile keeps t: no V(t)
+        const int vs = n % NV;
+        // the slot's previous load has been read by its PVs
+        if (n >= NV && !mbar_wait(&v_empty[vs], ((n / NV) - 1) & 1, fs)) break;
+        const int kb = kb_hi - t;
+        mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(&tm_v, &v_full[vs], sV + vs * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, k_off + kb * BK,
+                      bt);
+        if (p.v_tiles != nullptr) atomicAdd(p.v_tiles, 1ull);
+        ++n;
+      }
+      // loads the MMA thread may not have waited for (only after a wait gave up)
+      for (int i = max(0, n - NV); i < n; ++i) mbar_wait_drain(&v_full[i % NV], (i / NV) & 1);
     }
     __syncwarp();
   } else {
@@ -373,6 +440,12 @@ __global__ void __launch_bounds__(320, 1)
       const bool my_keep = qi == 0 ? bk0 : bk1;
       const bool need_pv = bk0 || bk1;
       if (tid == 0) {
+        if (kGate) {  // post the vote to the V issuer
+          reinterpret_cast<volatile uint32_t*>(vflag)[x * kVoteRing + t % kVoteRing] =
+              (need_pv ? 1u : 0u) | (any_abort ? 2u : 0u);
+          __threadfence_block();
+          reinterpret_cast<volatile uint32_t*>(vseq)[x] = static_cast<uint32_t>(t + 1);
+        }
         dec_flags[x] = (need_pv ? kDecPV : 0u) | (any_abort ? kDecAbort : 0u);
         mbar_arrive(&dec_bar[x]);
       }

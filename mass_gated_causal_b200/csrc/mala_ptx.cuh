@@ -3,9 +3,9 @@
 // and bounded waits.
 //
 // Every wait in this library is bounded: a wait that does not complete within
-// kWaitLimitNs sets the CTA's shared abort flag and the device status word,
-// and returns false so that the caller can leave its loop. No trap, no
-// unbounded spin.
+// its limit (kWaitLimitNs unless the host asked for another) sets the CTA's
+// shared abort flag and the device status word, and returns false so that
+// the caller can leave its loop. No trap, no unbounded spin.
 #pragma once
 
 #include <cuda.h>
@@ -80,6 +80,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 struct FailState {
   int* abort_flag;     // shared memory: set once any wait in the CTA gave up
   unsigned* status;    // global device status word
+  uint64_t limit_ns = kWaitLimitNs;  // how long one wait may take
 };
 
 __device__ __forceinline__ bool abort_raised(const FailState& fs) {
@@ -100,7 +101,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (mbar_try_wait_sleep(bar, parity)) return true;
     if ((n & 3u) == 0) {
       if (abort_raised(fs)) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > fs.limit_ns) {
         raise_abort(fs);
         return false;
       }
@@ -130,7 +131,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, c
       int give_up = 0;
       if ((threadIdx.x & 31) == 0) {
         give_up = abort_raised(fs) ? 1 : 0;
-        if (!give_up && global_timer_ns() - t0 > kWaitLimitNs) {
+        if (!give_up && global_timer_ns() - t0 > fs.limit_ns) {
           raise_abort(fs);
           give_up = 1;
         }

@@ -92,3 +92,44 @@ def test_fwd_batch2(cuda_lib):
 @pytest.mark.parametrize("w,tau", [(C1, 0.0), (C1, 1.0), (C1_IID, 0.0), (C1_IID, 1.0)])
 def test_fwd_c1(cuda_lib, w, tau):
     run_fwd_case(cuda_lib, w, tau)
+
+
+def pair_v_tiles(km, L, Bq):
+    """V tiles a gated forward loads: each CTA owns a pair of 128-row query tiles
+    of one (b, hq), and a key tile's V is loaded once if some query block of the
+    pair keeps it (agihunt.info MALA digest, method paragraphs: a skipped tile
+    does no V load)."""
+    B, H, nq, nk = km.shape
+    per = 256 // Bq
+    total = 0
+    for pr in range(-(-L // 256)):
+        blocks = list(range(pr * per, min((pr + 1) * per, nq)))
+        total += int((km[:, :, blocks, :] == 1).any(axis=2).sum())
+    return total
+
+
+@pytest.mark.parametrize("tau,Bq", [(1.0, 128), (16.0, 128), (16.0, 64)])
+def test_fwd_loads_v_only_for_kept_tiles(cuda_lib, tau, Bq):
+    mala = cuda_lib
+    L = 2048
+    w = TrainWorkload("vtiles", 1, 4, 2, L, 128, Bq, 128, seed=3300)
+    inp = make_train_inputs(w)
+    q, k, v = (_to_dev(inp[x]) for x in ("q", "k", "v"))
+    counter = torch.zeros(1, dtype=torch.int64, device="cuda")
+    assert mala.mala_test_hooks(0, -1, counter) == 0
+    try:
+        o, lse, kept, km = mala.forward(q, k, v, w.scale, tau, w.Bq, w.Bk, keep_map=True)
+        assert mala.mala_check_status() == 0
+    finally:
+        mala.mala_test_hooks(0, -1, None)
+    km_h = km.cpu().numpy()
+    ref = oracle.fwd(*(bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v")), w.scale, tau, w.Bq, w.Bk)
+    dec = compare_fwd_decisions(km_h, ref["keep"], ref["margin"], L, w.Bq, w.Bk)
+    assert dec["bad"] == 0, dec["bad_sites"][:10]
+    loaded = int(counter.item())
+    assert loaded == pair_v_tiles(km_h, L, w.Bq)
+    # key tiles the CTAs walk: kb = 0 .. the tile of the pair's last row
+    visits = w.B * w.Hq * sum((min(pr * 256 + 256, L) - 1) // w.Bk + 1 for pr in range(-(-L // 256)))
+    print(f"[fwd V tiles] tau={tau} Bq={Bq}: loaded {loaded} of {visits} walked")
+    if tau >= 16:
+        assert loaded < 0.9 * visits
