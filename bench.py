@@ -39,7 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import C2, C3, C4, C5, WORKLOADS, default_workers  # noqa: E402
+from workloads import C1, C1_IID, C2, C3, C4, C5, WORKLOADS, default_workers  # noqa: E402
 
 METRIC = "MALA fwd+bwd ms & eff. TFLOP/s (% bf16 peak) at 32K/128K, τ=1; retained-tile %"
 L2_BYTES = 126 * 1024 * 1024
@@ -177,6 +177,13 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CUDA arm
 # --------------------------------------------------------------------------
+def bench_config(w, tau, world):
+    """The `config` object of the JSON line (identical in both arms)."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d, "Bq": w.Bq, "Bk": w.Bk,
+            "tau": tau, "scale": w.scale, "seed": w.seed, "parallelism": f"replicas x{world} (head slices)",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
 def _dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -326,6 +333,30 @@ def run_cuda(args):
     ms0_b = max_over_ranks(float(np.mean(b0)))
     flops0 = fl0["fwd"] + fl0["bwd"]
 
+    # larger tau on the same inputs: how the step time follows the retained work
+    sweep = {}
+    for tau_s in (4.0, 16.0):
+        km_f = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8, device=dev)
+        km_b = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8, device=dev)
+        step(tau_s, km_f, km_b)
+        assert mala.mala_check_status(stream) == 0
+        kf_s, kb_s = km_f.cpu().numpy(), km_b.cpu().numpy()
+        del km_f, km_b
+        fl_s = train_flops(d, B, Hq, L, live, kf_s, kb_s)
+        tot_s, f_s, b_s = timed(train_step(tau_s), 3, 3)
+        ms_s = max_over_ranks(float(np.mean(tot_s)))
+        sweep[f"tau{int(tau_s)}"] = {
+            "ms_per_step": round(ms_s, 3), "fwd_ms": round(max_over_ranks(float(np.mean(f_s))), 3),
+            "bwd_ms": round(max_over_ranks(float(np.mean(b_s))), 3),
+            "tflops": round(world * (fl_s["fwd"] + fl_s["bwd"]) / (ms_s * 1e-3) / 1e12, 2),
+            "retained_tiles_fwd": round(float((kf_s == 1).sum() / (legal.sum() * B * Hq)), 4),
+            "retained_tiles_bwd": round(float((kb_s == 1).sum() / (legal.sum() * B * Hq)), 4),
+            "speedup_vs_tau0": round(ms0 / ms_s, 3)}
+    assert mala.mala_check_status(stream) == 0
+
+    # matched work (the pages' fidelity comparison) on the CUDA forward's keep map
+    mw = matched_work_sample(torch, dev, q, k, v, kmf, w, n_blocks=8, seed=w.seed + 600)
+
     # e2e through the C ABI from pinned host buffers
     hq_, hk_, hv_, hdo_ = (torch.from_numpy(inp[x].view(np.int16)).view(torch.bfloat16).pin_memory()
                            for x in ("q", "k", "v", "do"))
@@ -398,17 +429,26 @@ def run_cuda(args):
     # the same fwd+bwd step on the 128K workload (the metric is quoted at 32K and 128K)
     long_leg = None
     if not args.no_long and w.name != C3.name:
-        long_leg = run_train_leg(C3, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world)
+        long_leg = run_train_leg(C3, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world,
+                                 oracle_seconds=0.0 if (args.no_cpu or rank != 0 or world > 1) else 8.0)
 
     # a packed batch of mixed lengths (32K tokens in all)
     varlen_leg = None
     if not args.no_varlen:
         varlen_leg = run_varlen_leg(C5, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world)
 
+    # the 8K workloads (structured and diffuse inputs): gate overhead in the low-skip regime
+    legs_8k = None
+    if not args.no_8k:
+        legs_8k = {x.name: run_train_leg(x, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world,
+                                         oracle_seconds=0.0 if (args.no_cpu or rank != 0 or world > 1) else 3.0)
+                   for x in (C1, C1_IID)}
+
     # decode workload
     dec = None
     if not args.no_decode:
-        dec = run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world)
+        dec = run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world,
+                         oracle_seconds=0.0 if (args.no_cpu or rank != 0 or world > 1) else 8.0)
 
     # roofline of the dominant kernel (fwd or bwd call, timed with events on its stream)
     peak_t = pk["bf16_tflops_sustained"]
@@ -433,9 +473,7 @@ def run_cuda(args):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded structured generator)",
-        "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "L": L, "d": d, "Bq": w.Bq, "Bk": w.Bk,
-                   "tau": tau, "scale": w.scale, "seed": w.seed, "parallelism": f"replicas x{world} (head slices)",
-                   "l2": "inputs larger than L2 (no flush)"},
+        "config": bench_config(w, tau, world),
         "frac_of_peak": round(value / world / peak_t, 4),
         "retained_tiles": {"fwd_mean": round(float(kept_frac_f.mean()), 4),
                            "fwd_min": round(float(kept_frac_f.min()), 4),
@@ -446,6 +484,8 @@ def run_cuda(args):
                            "live_pair_frac_fwd": round(fl["n_f"] / fl["n_legal"], 4),
                            "live_pair_frac_bwd": round(fl["n_b"] / fl["n_legal"], 4)},
         "fwd_ms": round(ms_f, 3), "bwd_ms": round(ms_b, 3), "step_tflop": round(step_flops / 1e12, 3),
+        "tau0_ms_per_step": round(ms0, 3), "mala_speedup": round(ms0 / ms,  3),
+        "tau_sweep": sweep, "matched_work": mw,
         "fullattn_tau0": {"ms_per_step": round(ms0, 3), "fwd_ms": round(ms0_f, 3), "bwd_ms": round(ms0_b, 3),
                           "tflops": round(world * flops0 / (ms0 * 1e-3) / 1e12, 3),
                           "frac_of_peak": round(flops0 / (ms0 * 1e-3) / 1e12 / peak_t, 4),
@@ -463,6 +503,8 @@ def run_cuda(args):
         line["at_128k"] = long_leg
     if varlen_leg is not None:
         line["varlen"] = varlen_leg
+    if legs_8k is not None:
+        line["at_8k"] = legs_8k
     if dec is not None:
         line["decode"] = dec
     if cpu is not None:
@@ -475,13 +517,14 @@ def run_cuda(args):
         dist.destroy_process_group()
 
 
-def run_train_leg(w, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world, steps=3, warmup=3):
-    """fwd+bwd at tau = 1 and tau = 0 on workload `w` (ms, effective TFLOP/s, retained tiles)."""
+def run_train_leg(w, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world, steps=3, warmup=3,
+                  oracle_seconds=0.0):
+    """fwd+bwd at tau = 1 and tau = 0 on workload `w` (ms, effective TFLOP/s, retained tiles); with
+    oracle_seconds > 0 also the CPU oracle on a seeded sample of query blocks, with the full run extrapolated."""
     from workloads import make_train_inputs
     inp = make_train_inputs(w, workers=workers)
     to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
     q, k, v, do = (to_dev(inp[x]) for x in ("q", "k", "v", "do"))
-    del inp
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     o = torch.empty_like(q)
@@ -533,6 +576,9 @@ def run_train_leg(w, mala, torch, dev, stream, pk, workers, timed, max_over_rank
                     "frac_of_peak": round(tf / world / peak_t, 4)}
     assert mala.mala_check_status(stream) == 0
     out["mala_speedup"] = round(out["tau0"]["ms_per_step"] / out["tau1"]["ms_per_step"], 3)
+    if oracle_seconds > 0:
+        out["oracle"] = oracle_subset(w, inp, 1.0, oracle_seconds, fl["fwd"] + fl["bwd"])
+    del inp
     return out
 
 
@@ -646,7 +692,7 @@ def run_paged_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, 
     return out
 
 
-def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world):
+def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_ranks, world, oracle_seconds=0.0):
     from workloads import make_decode_inputs
     w = C4
     inp = make_decode_inputs(w, workers=workers)
@@ -691,6 +737,8 @@ def run_decode(args, mala, torch, dev, stream, pk, workers, timed, max_over_rank
     out["hbm_peak_gbs"] = pk["hbm_gbs"]
     out["paged"] = run_paged_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, out)
     out["exact"] = run_exact_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, q, kc, vc, w, out)
+    if oracle_seconds > 0:
+        out["oracle"] = oracle_decode_subset(w, inp, 1.0, ns, oracle_seconds, out["tau1"]["us_per_step"])
     return out
 
 
@@ -738,6 +786,62 @@ def run_exact_decode(args, mala, torch, dev, stream, pk, timed, max_over_ranks, 
                     "vs_split_decode": round(contiguous[key]["us_per_step"] / us, 3)}
     assert mala.mala_check_status(stream) == 0
     return out
+
+
+def matched_work_sample(torch, dev, q, k, v, keep_map, w, n_blocks, seed):
+    """The pages' matched-work comparison (agihunt.info MALA digest, fidelity
+    paragraphs) on a seeded sample of query blocks, from the CUDA forward's keep
+    map: per row, MALA's key slots (the live keys of its kept tiles), its omitted
+    probability mass and output error against dense attention, and the same for
+    the reference-mass policy given the same number of slots (the row's largest
+    probabilities). MALA's output is the softmax over its retained keys, which is
+    what the forward computes up to rounding. fp64 on the GPU with torch: a
+    diagnostic beside the measurement, not part of the operator."""
+    rng = np.random.default_rng(seed)
+    B, L, Hq, d = q.shape
+    G = Hq // k.shape[2]
+    nq = keep_map.shape[2]
+    acc = {x: [] for x in ("slots", "live", "omit_mala", "omit_ref", "err_mala", "err_ref")}
+    ar = torch.arange(L, device=dev)
+    sample = []
+    for _ in range(n_blocks):
+        b, h, qb = int(rng.integers(B)), int(rng.integers(Hq)), int(rng.integers(nq))
+        sample.append((b, h, qb))
+        rows = torch.arange(qb * w.Bq, min((qb + 1) * w.Bq, L), device=dev)
+        kk, vv = k[b, :, h // G].double(), v[b, :, h // G].double()
+        live = ar[None, :] <= rows[:, None]
+        sc = (q[b, rows, h].double() @ kk.T) * w.scale
+        p = torch.softmax(sc.masked_fill(~live, float("-inf")), dim=1)
+        o_dense = p @ vv
+        kept_keys = torch.from_numpy(np.repeat(keep_map[b, h, qb] == 1, w.Bk)[:L].copy()).to(dev)
+        ret = live & kept_keys[None, :]
+        slots = ret.sum(1)
+        pm = p * ret
+        omit_mala = 1.0 - pm.sum(1)
+        o_mala = (pm @ vv) / pm.sum(1, keepdim=True)
+        order = torch.argsort(p, dim=1, descending=True, stable=True)
+        rank = torch.empty_like(order)
+        rank.scatter_(1, order, ar[None, :].expand(len(rows), L).contiguous())
+        pr = torch.where(rank < slots[:, None], p, torch.zeros_like(p))
+        omit_ref = 1.0 - pr.sum(1)
+        o_ref = (pr @ vv) / pr.sum(1, keepdim=True)
+        nrm = o_dense.norm(dim=1)
+        for key_, val in (("slots", slots), ("live", live.sum(1)), ("omit_mala", omit_mala), ("omit_ref", omit_ref),
+                          ("err_mala", (o_mala - o_dense).norm(dim=1) / nrm),
+                          ("err_ref", (o_ref - o_dense).norm(dim=1) / nrm)):
+            acc[key_].append(val.double().cpu().numpy())
+        del sc, p, pm, pr, order, rank
+    r = {x: np.concatenate(v_) for x, v_ in acc.items()}
+    return {"rows": int(r["slots"].size), "blocks": n_blocks, "tau": 1.0,
+            "slot_frac": round(float(r["slots"].sum() / r["live"].sum()), 4),
+            "slots_per_query_mean": round(float(r["slots"].mean()), 1),
+            "omitted_mass_mala_mean": float(f"{r['omit_mala'].mean():.4g}"),
+            "omitted_mass_ref_mean": float(f"{r['omit_ref'].mean():.4g}"),
+            "omitted_mass_mala_max": float(f"{r['omit_mala'].max():.4g}"),
+            "out_rel_err_mala_mean": float(f"{r['err_mala'].mean():.4g}"),
+            "out_rel_err_ref_mean": float(f"{r['err_ref'].mean():.4g}"),
+            "keep_map": "CUDA forward (the diagnostic pass)", "precision": "fp64 (torch on the GPU)",
+            "sample": f"{n_blocks} seeded query blocks (b, hq, qb): {sample}"}
 
 
 # --------------------------------------------------------------------------
@@ -791,6 +895,54 @@ def cpu_baseline(w, inp, tau, seconds):
                                         f"the backward, {flops / 1e9:.1f} GFLOP effective in {dt:.1f} s"}
 
 
+def oracle_subset(w, inp, tau, seconds, full_flops):
+    """The oracle on a seeded sample of query blocks (forward + dQ part of the
+    backward), grown to about `seconds` of host time; the full fwd+bwd run is
+    extrapolated by effective FLOPs (the sample's against the whole step's)."""
+    import oracle
+    from workloads import bf16_bits_to_f64
+    qf, kf, vf, dof = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v", "do"))
+    n = 2
+    while True:
+        sel = oracle_sample(w, inp, tau, n, seed=w.seed + 500)
+        flops, dt = run_oracle_sample(w, qf, kf, vf, dof, tau, sel)
+        if dt >= seconds / 3 or n >= 1024:
+            break
+        n *= 2
+    return {"kind": "oracle", "cores": oracle.num_threads(), "subset_blocks": len(sel),
+            "subset_ms": round(dt * 1e3, 1), "subset_gflop": round(flops / 1e9, 2),
+            "tflops": round(flops / dt / 1e12, 6),
+            "extrapolated_full_step_ms": round(dt * 1e3 * full_flops / flops, 0),
+            "sample": f"{len(sel)} seeded query blocks of {w.name}: forward + dQ part of the backward; the full "
+                      f"step is extrapolated by effective FLOPs"}
+
+
+def oracle_decode_subset(w, inp, tau, n_splits, seconds, full_us):
+    """The oracle's decode on a seeded sample of (b, query head) rows, grown to
+    about `seconds`; the full step is extrapolated by rows."""
+    import oracle
+    from workloads import bf16_bits_to_f64
+    rng = np.random.default_rng(w.seed + 500)
+    b0 = int(rng.integers(0, w.B))  # one sequence's cache in fp64 (about 2 GB at 128K) bounds host memory
+    qf, kf, vf = (bf16_bits_to_f64(inp[x][b0:b0 + 1]) for x in ("q", "kcache", "vcache"))
+    rows_all = [(0, h) for h in range(w.Hq)]
+    n = 2
+    while True:
+        idx = rng.permutation(len(rows_all))[:n]
+        sel = [rows_all[i] for i in idx]
+        t0 = time.perf_counter()
+        oracle.decode(qf, kf, vf, w.scale, tau, w.Bk, n_splits, sel=sel)
+        dt = time.perf_counter() - t0
+        if dt >= seconds / 3 or n >= len(rows_all):
+            break
+        n = min(2 * n, len(rows_all))
+    full_ms = dt * 1e3 * w.B * w.Hq / len(sel)
+    return {"kind": "oracle", "cores": oracle.num_threads(), "subset_rows": len(sel), "subset_ms": round(dt * 1e3, 1),
+            "extrapolated_full_step_ms": round(full_ms, 1), "gpu_speedup": round(full_ms * 1e3 / full_us, 1),
+            "sample": f"{len(sel)} seeded (b, query head) rows of {w.name} (split decode, same split count); the "
+                      f"full step is extrapolated by rows"}
+
+
 def run_reference(args):
     world, rank, _ = _dist_env()
     if rank != 0:
@@ -815,8 +967,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(times)), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded structured generator)",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d, "Bq": w.Bq,
-                       "Bk": w.Bk, "tau": tau},
+            "config": bench_config(w, tau, world),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                              "kind": "oracle",
                              "sample": f"each step: {n} seeded query blocks of {w.name}, forward + dQ part "
@@ -920,6 +1071,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the 128K fwd+bwd leg")
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch fwd+bwd leg")
+    ap.add_argument("--no-8k", action="store_true", help="skip the 8K structured / diffuse fwd+bwd legs")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-blocks", type=int, default=16)

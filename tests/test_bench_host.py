@@ -88,3 +88,40 @@ def test_packed_flops_sum_per_sequence():
                     want += int(km[s, h, i // Bt, j // Bt] == 1)
     assert fl["n_f"] == fl["n_b"] == want
     assert fl["fwd"] == 2 * d * tri + 2 * d * want and fl["bwd"] == 2 * d * tri + 8 * d * want
+
+
+def test_matched_work_sample_equals_the_oracle_analysis():
+    # the bench's torch fp64 matched-work diagnostic (run on the GPU there) gives,
+    # on the CPU, the per-row figures of oracle/matched_work.py for the same keep map
+    import math
+
+    import torch
+
+    from oracle import fwd
+    from oracle.matched_work import matched_work
+    from workloads import TrainWorkload, bf16_bits_to_f64, make_train_inputs
+
+    w = TrainWorkload("mw_host", 1, 2, 1, 300, 32, 16, 16, seed=9100)
+    inp = make_train_inputs(w)
+    qf, kf, vf = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v"))
+    keep = fwd(qf, kf, vf, w.scale, 1.0, w.Bq, w.Bk)["keep"]
+    t = lambda a: torch.from_numpy(a)
+    out = bench.matched_work_sample(torch, "cpu", t(qf), t(kf), t(vf), keep, w, n_blocks=6, seed=5)
+    blocks = [tuple(int(x) for x in s.strip("() ").split(",")) for s in
+              out["sample"].split(": ", 1)[1].strip("[]").split("), (")]
+    ref = matched_work(qf, kf, vf, w.scale, 1.0, w.Bq, w.Bk, keep=keep)
+    nq = -(-w.L // w.Bq)
+    rows = np.concatenate([np.arange(h * w.L + qb * w.Bq, h * w.L + min((qb + 1) * w.Bq, w.L))
+                           for (b, h, qb) in blocks])
+    assert out["rows"] == rows.size
+    assert math.isclose(out["slot_frac"], round(ref["slots"][rows].sum() / ref["live"][rows].sum(), 4))
+    for key, name in (("omitted_mass_mala_mean", "omit_mala"), ("omitted_mass_ref_mean", "omit_ref"),
+                      ("out_rel_err_mala_mean", "err_mala"), ("out_rel_err_ref_mean", "err_ref")):
+        assert math.isclose(out[key], ref[name][rows].mean(), rel_tol=1e-3, abs_tol=1e-12), key
+    assert nq == keep.shape[2]
+
+
+def test_both_arms_report_the_same_config():
+    from workloads import C2
+    a = bench.bench_config(C2, 1.0, 1)
+    assert a == bench.bench_config(C2, 1.0, 1) and a["workload"] == C2.name and a["tau"] == 1.0
