@@ -103,3 +103,17 @@ def test_decode_small(cuda_lib, Lk, d, Bk, tau, n_splits):
 def test_decode_gqa8(cuda_lib):
     w = DecodeWorkload("dec_gqa8", 1, 16, 2, 3000, 128, 128, seed=5101)
     run_decode_case(cuda_lib, w, 1.0, n_splits=4)
+
+
+@pytest.mark.parametrize("Hq,Hkv,Lk,d,Bk,tau,n_splits", [
+    (4, 2, 2500, 128, 128, 1.0, 3),    # two heads per group: one (key, head) value per lane
+    (6, 2, 2500, 128, 128, 1.0, 2),    # three heads padded to four
+    (4, 2, 1500, 64, 128, 0.5, 3),     # d = 64
+    (6, 2, 900, 64, 64, 2.0, 2),       # d = 64, 64-key tiles, padded heads
+])
+def test_decode_group_sizes(cuda_lib, Hq, Hkv, Lk, d, Bk, tau, n_splits):
+    """Group sizes and tile shapes of the batched scoring: the (step, head) dot
+    products of a tile are reduced together and each lane keeps one or two of
+    them; padded heads take part in the reduction and are never gated."""
+    w = DecodeWorkload("dec_groups", 2, Hq, Hkv, Lk, d, Bk, seed=5200 + Hq + Lk + d)
+    run_decode_case(cuda_lib, w, tau, n_splits=n_splits)
