@@ -16,7 +16,7 @@
 // mala_bwd_kernel: one CTA owns 128 keys (one key block when Bk = 128, two
 // when Bk = 64) of one (b, KV head) and walks the query tiles of every query
 // head of the GQA group, 128 queries at a time, from the diagonal tile to the
-// last, one head after the other. dK and dV accumulate in
+// last, each tile for all heads of the group in turn. dK and dV accumulate in
 // TMEM across the whole walk. 14 warps:
 //   warps 0-7   compute: thread t owns query row t % 128 of the current tile
 //               and key columns [64h, 64h + 64), h = t / 128 (TMEM lane row of
@@ -171,12 +171,16 @@ __global__ void __launch_bounds__(448, 1)
   const int k0 = ks * 128;
   const int nqs = n_super - ks;
   const int T = p.G * nqs;
-  // Walk order: the G query heads one after the other, each from the diagonal
-  // query tile to the last. (Walking every CTA of a KV head through the same
-  // tiles in step was measured slower: their dQ additions then hit the same
-  // lines at once.) The backward decisions do not depend on the order.
-  auto walk_hq = [&](int t) { return hkv * p.G + t / nqs; };
-  auto walk_qs = [&](int t) { return ks + t % nqs; };
+  // Walk order: query tiles from the diagonal to the last, and for each the G
+  // query heads of the group in turn, so the CTAs of a KV head move through
+  // the query rows G times slower and their Q / dO / dQ lines stay in L2
+  // longer (1-3% faster than one head after the other, measured at 32K GQA
+  // across tau). Walking every CTA of a KV head through the same tiles in
+  // step was measured slower (their dQ additions then hit the same lines at
+  // once), and so were staggered groups. The backward decisions do not depend
+  // on the order.
+  auto walk_hq = [&](int t) { return hkv * p.G + t % p.G; };
+  auto walk_qs = [&](int t) { return ks + t / p.G; };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
