@@ -90,6 +90,17 @@ def packed_flops(lens, Hq, d, Bq, Bk, keep_f, keep_b):
     return fl
 
 
+def pair_v_tiles(km, L: int, Bq: int) -> int:
+    """V tiles the default forward loads: a CTA owns a pair of 128-row query
+    tiles of one (b, hq) and loads a key tile's V once if some query block of
+    the pair keeps it."""
+    km = np.asarray(km)
+    per = 256 // Bq
+    nq = km.shape[2]
+    return int(sum((km[:, :, pr * per:min((pr + 1) * per, nq), :] == 1).any(axis=2).sum()
+                   for pr in range(-(-L // 256))))
+
+
 def decode_bytes(B, Hq, Hkv, Lk, d, Bk, keep_map):
     """Algorithmic bytes of one decode step: all K, V of tiles kept by >= 1 head of
     the group, q in and o out (bf16)."""
@@ -335,12 +346,14 @@ def run_cuda(args):
 
     # larger tau on the same inputs: how the step time follows the retained work
     sweep = {}
+    km_by_tau = {tau: kmf}
     for tau_s in (4.0, 16.0):
         km_f = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8, device=dev)
         km_b = torch.zeros((B, Hq, nq, nk), dtype=torch.uint8, device=dev)
         step(tau_s, km_f, km_b)
         assert mala.mala_check_status(stream) == 0
         kf_s, kb_s = km_f.cpu().numpy(), km_b.cpu().numpy()
+        km_by_tau[tau_s] = kf_s
         del km_f, km_b
         fl_s = train_flops(d, B, Hq, L, live, kf_s, kb_s)
         tot_s, f_s, b_s = timed(train_step(tau_s), 3, 3)
@@ -352,6 +365,30 @@ def run_cuda(args):
             "retained_tiles_fwd": round(float((kf_s == 1).sum() / (legal.sum() * B * Hq)), 4),
             "retained_tiles_bwd": round(float((kb_s == 1).sum() / (legal.sum() * B * Hq)), 4),
             "speedup_vs_tau0": round(ms0 / ms_s, 3)}
+    assert mala.mala_check_status(stream) == 0
+
+    # the opt-in V prefetch (mala_fwd_ex, MALA_FWD_PREFETCH_V: every V tile fetched
+    # ahead of the vote) against the default (V requested only for kept tiles):
+    # the forward alone, same inputs and decisions
+    def fwd_only(tau_, flags):
+        def fn(mid=None):
+            rc = mala.mala_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, L, d, w.scale, tau_, w.Bq, w.Bk, fws, fws_bytes,
+                                  kept_f, None, stream, flags)
+            assert rc == 0
+            if mid is not None:
+                mid.record(stream)
+        return fn
+
+    prefetch = {}
+    walked = B * Hq * sum((min(pr * 256 + 256, L) - 1) // w.Bk + 1 for pr in range(-(-L // 256)))
+    for tau_p in sorted(km_by_tau):
+        t_dem, _, _ = timed(fwd_only(tau_p, 0), 5, 3)
+        t_pre, _, _ = timed(fwd_only(tau_p, mala.MALA_FWD_PREFETCH_V), 5, 3)
+        ms_dem, ms_pre = max_over_ranks(float(np.mean(t_dem))), max_over_ranks(float(np.mean(t_pre)))
+        prefetch[f"tau{tau_p:g}"] = {
+            "fwd_ms_v_on_demand": round(ms_dem, 3), "fwd_ms_v_prefetched": round(ms_pre, 3),
+            "v_tiles_on_demand_frac": round(pair_v_tiles(km_by_tau[tau_p], L, w.Bq) / walked, 4),
+            "v_tiles_prefetched_frac": 1.0}
     assert mala.mala_check_status(stream) == 0
 
     # matched work (the pages' fidelity comparison) on the CUDA forward's keep map
@@ -485,7 +522,7 @@ def run_cuda(args):
                            "live_pair_frac_bwd": round(fl["n_b"] / fl["n_legal"], 4)},
         "fwd_ms": round(ms_f, 3), "bwd_ms": round(ms_b, 3), "step_tflop": round(step_flops / 1e12, 3),
         "tau0_ms_per_step": round(ms0, 3), "mala_speedup": round(ms0 / ms,  3),
-        "tau_sweep": sweep, "matched_work": mw,
+        "tau_sweep": sweep, "fwd_prefetch_v": prefetch, "matched_work": mw,
         "fullattn_tau0": {"ms_per_step": round(ms0, 3), "fwd_ms": round(ms0_f, 3), "bwd_ms": round(ms0_b, 3),
                           "tflops": round(world * flops0 / (ms0 * 1e-3) / 1e12, 3),
                           "frac_of_peak": round(flops0 / (ms0 * 1e-3) / 1e12 / peak_t, 4),

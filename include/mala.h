@@ -103,6 +103,25 @@ MALA_API int mala_fwd(const void* q, const void* k, const void* v, void* o, floa
              size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream);
 
 /*
+ * mala_fwd_ex -- mala_fwd with option flags (flags = 0 is exactly mala_fwd).
+ *
+ *   MALA_FWD_PREFETCH_V  fetch the V tile of every legal key tile ahead of
+ *            the gate's decision instead of only after a query block has
+ *            voted to keep it. The keep/skip decisions, O, LSE, kept_tiles
+ *            and keep_map are the same as without the flag; a skipped tile
+ *            still gets no softmax update and no PV, but its V tile is read
+ *            (the digest's method paragraphs list the V load among the work a
+ *            skip saves, so this is a departure from the method's cost model,
+ *            offered because no PV then waits for a V load requested after a
+ *            vote). Without tau > 0 the flag changes nothing.
+ * Errors: as mala_fwd; MALA_ERR_INVALID_ARG also for an unknown flag bit.
+ */
+#define MALA_FWD_PREFETCH_V 1u
+MALA_API int mala_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int L, int d, float scale, float tau, int Bq, int Bk, void* workspace,
+             size_t workspace_bytes, int32_t* kept_tiles, uint8_t* keep_map, void* stream, unsigned flags);
+
+/*
  * Workspace bytes mala_fwd needs: the fp16 copy of V [B, L, Hkv, d] the PV
  * product reads (256-byte aligned). Returns 0 for invalid sizes. mala_prefill
  * needs mala_fwd_workspace_size(B, Hkv, Lk, d).

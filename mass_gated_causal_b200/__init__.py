@@ -34,8 +34,9 @@ MALA_ERR_WORKSPACE = 3
 MALA_ERR_CUDA = 4
 MALA_ERR_DEVICE_TIMEOUT = 5
 MALA_ERR_RANGE = 6
+MALA_FWD_PREFETCH_V = 1
 
-EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_prefill", "mala_fwd_varlen",
+EXPORTED = ("mala_status_string", "mala_abi_version", "mala_fwd", "mala_fwd_ex", "mala_prefill", "mala_fwd_varlen",
             "mala_fwd_workspace_size", "mala_bwd_workspace_size", "mala_bwd", "mala_bwd_varlen",
             "mala_decode_workspace_size", "mala_decode_default_splits", "mala_decode", "mala_decode_paged",
             "mala_decode_exact_workspace_size", "mala_decode_exact",
@@ -47,6 +48,9 @@ _lib.mala_status_string.restype = ctypes.c_char_p
 _lib.mala_abi_version.restype = _i
 _lib.mala_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp, _vp]
 _lib.mala_fwd.restype = _i
+_lib.mala_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp, _vp,
+                             ctypes.c_uint]
+_lib.mala_fwd_ex.restype = _i
 _lib.mala_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _f, _i, _i, _vp, _sz, _vp, _vp,
                               _vp]
 _lib.mala_prefill.restype = _i
@@ -130,6 +134,13 @@ def mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace, w
     return int(_lib.mala_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), B, Hq, Hkv, L, d, float(scale), float(tau),
                              Bq, Bk, _p(workspace), int(workspace_bytes), _p(kept_tiles), _p(keep_map),
                              _stream(stream)))
+
+
+def mala_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace, workspace_bytes, kept_tiles,
+                keep_map=None, stream=None, flags=0) -> int:
+    return int(_lib.mala_fwd_ex(_p(q), _p(k), _p(v), _p(o), _p(lse), B, Hq, Hkv, L, d, float(scale), float(tau),
+                                Bq, Bk, _p(workspace), int(workspace_bytes), _p(kept_tiles), _p(keep_map),
+                                _stream(stream), int(flags)))
 
 
 def mala_prefill(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, tau, Bq, Bk, workspace, workspace_bytes,
@@ -227,8 +238,10 @@ def mala_check_status(stream=None) -> int:
 
 # ------------------------------------------------------------ conveniences
 def forward(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, keep_map: bool = False,
-            workspace=None, stream=None):
-    """q [B,L,Hq,d], k/v [B,L,Hkv,d] bf16 CUDA tensors -> (o, lse, kept_tiles, keep_map|None)."""
+            workspace=None, stream=None, prefetch_v: bool = False):
+    """q [B,L,Hq,d], k/v [B,L,Hkv,d] bf16 CUDA tensors -> (o, lse, kept_tiles, keep_map|None).
+
+    prefetch_v: fetch every V tile ahead of the gate (mala_fwd_ex with MALA_FWD_PREFETCH_V)."""
     import torch
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -240,8 +253,9 @@ def forward(q, k, v, scale: float, tau: float, Bq: int = 128, Bk: int = 128, kee
     km = None
     if keep_map:
         km = torch.full((B, Hq, -(-L // Bq), -(-L // Bk)), 255, dtype=torch.uint8, device=q.device)
-    _check(mala_fwd(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace,
-                    workspace.numel() * workspace.element_size(), kept, km, stream), "mala_fwd")
+    _check(mala_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, L, d, scale, tau, Bq, Bk, workspace,
+                       workspace.numel() * workspace.element_size(), kept, km, stream,
+                       MALA_FWD_PREFETCH_V if prefetch_v else 0), "mala_fwd")
     return o, lse, kept, km
 
 

@@ -131,11 +131,11 @@ int fwd_chunk_pairs(int n_pairs, int G) {
 int bwd_chunk_kb(int n_super) { return std::max(1, std::min(sm_count(), (n_super + 1) / 2)); }
 
 // ---------------------------------------------------------------- forward
-template <int D, int BQ, int BK, bool G>
+template <int D, int BQ, int BK, int MODE>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                const mala::FwdParams& p, cudaStream_t st) {
   using Lay = mala::FwdLayout<D, BK>;
-  auto kern = mala::mala_fwd_kernel<D, BQ, BK, G>;
+  auto kern = mala::mala_fwd_kernel<D, BQ, BK, MODE>;
   if (set_smem(kern, Lay::ALLOC_BYTES) != MALA_OK) return MALA_ERR_CUDA;
   const unsigned n_chunks = (p.n_pairs + p.chunk_pairs - 1) / p.chunk_pairs;
   const unsigned grid = n_chunks * p.chunk_pairs * p.B * p.Hq;
@@ -143,20 +143,22 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
+// mode: 0 no gate, 1 gate with V on demand, 2 gate with V fetched ahead
 template <int D, int BQ, int BK>
-int launch_fwd_gate(bool gate, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+int launch_fwd_gate(int mode, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mo, const mala::FwdParams& p, cudaStream_t st) {
-  return gate ? launch_fwd<D, BQ, BK, true>(mq, mk, mv, mo, p, st)
-              : launch_fwd<D, BQ, BK, false>(mq, mk, mv, mo, p, st);
+  if (mode == 1) return launch_fwd<D, BQ, BK, 1>(mq, mk, mv, mo, p, st);
+  if (mode == 2) return launch_fwd<D, BQ, BK, 2>(mq, mk, mv, mo, p, st);
+  return launch_fwd<D, BQ, BK, 0>(mq, mk, mv, mo, p, st);
 }
 
 template <int D>
-int launch_fwd_tiles(int Bq, int Bk, bool gate, const CUtensorMap& mq, const CUtensorMap& mk,
+int launch_fwd_tiles(int Bq, int Bk, int mode, const CUtensorMap& mq, const CUtensorMap& mk,
                      const CUtensorMap& mv, const CUtensorMap& mo, const mala::FwdParams& p, cudaStream_t st) {
-  if (Bq == 128 && Bk == 128) return launch_fwd_gate<D, 128, 128>(gate, mq, mk, mv, mo, p, st);
-  if (Bq == 64 && Bk == 64) return launch_fwd_gate<D, 64, 64>(gate, mq, mk, mv, mo, p, st);
-  if (Bq == 64 && Bk == 128) return launch_fwd_gate<D, 64, 128>(gate, mq, mk, mv, mo, p, st);
-  return launch_fwd_gate<D, 128, 64>(gate, mq, mk, mv, mo, p, st);
+  if (Bq == 128 && Bk == 128) return launch_fwd_gate<D, 128, 128>(mode, mq, mk, mv, mo, p, st);
+  if (Bq == 64 && Bk == 64) return launch_fwd_gate<D, 64, 64>(mode, mq, mk, mv, mo, p, st);
+  if (Bq == 64 && Bk == 128) return launch_fwd_gate<D, 64, 128>(mode, mq, mk, mv, mo, p, st);
+  return launch_fwd_gate<D, 128, 64>(mode, mq, mk, mv, mo, p, st);
 }
 
 // --------------------------------------------------------------- backward
@@ -283,7 +285,8 @@ struct Packed {
 // packed batch, B counts the sequences and Lq / Lk are the longest lengths.
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
             int Lk, int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
-            int32_t* kept_tiles, uint8_t* keep_map, void* stream, const Packed& pk = Packed()) {
+            int32_t* kept_tiles, uint8_t* keep_map, void* stream, const Packed& pk = Packed(),
+            bool prefetch_v = false) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return MALA_ERR_UNSUPPORTED;
   const bool packed = pk.cu_q != nullptr;
@@ -326,9 +329,9 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   mala::mala_v_to_f16_kernel<<<cv_grid, 256, 0, st>>>(static_cast<const uint4*>(v), static_cast<uint4*>(workspace),
                                                       n8, status);
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
-  const bool gate = tau > 0.f;
-  if (d == 128) return launch_fwd_tiles<128>(Bq, Bk, gate, mq, mk, mv, mo, p, st);
-  return launch_fwd_tiles<64>(Bq, Bk, gate, mq, mk, mv, mo, p, st);
+  const int mode = tau > 0.f ? (prefetch_v ? 2 : 1) : 0;
+  if (d == 128) return launch_fwd_tiles<128>(Bq, Bk, mode, mq, mk, mv, mo, p, st);
+  return launch_fwd_tiles<64>(Bq, Bk, mode, mq, mk, mv, mo, p, st);
 }
 }  // namespace
 
@@ -340,6 +343,17 @@ int mala_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (rc != MALA_OK) return rc;
   return run_fwd(q, k, v, o, lse, B, Hq, Hkv, L, L, d, scale, tau, Bq, Bk, workspace, workspace_bytes, kept_tiles,
                  keep_map, stream);
+}
+
+int mala_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int L,
+                int d, float scale, float tau, int Bq, int Bk, void* workspace, size_t workspace_bytes,
+                int32_t* kept_tiles, uint8_t* keep_map, void* stream, unsigned flags) {
+  if (!q || !k || !v || !o || !lse || !kept_tiles) return MALA_ERR_INVALID_ARG;
+  if (flags & ~MALA_FWD_PREFETCH_V) return MALA_ERR_INVALID_ARG;
+  int rc = check_train_shape(B, Hq, Hkv, L, d, scale, tau, Bq, Bk);
+  if (rc != MALA_OK) return rc;
+  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, L, L, d, scale, tau, Bq, Bk, workspace, workspace_bytes, kept_tiles,
+                 keep_map, stream, Packed(), (flags & MALA_FWD_PREFETCH_V) != 0);
 }
 
 int mala_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,

@@ -20,9 +20,10 @@
 //   warps 0-3  softmax warpgroup of tile A (thread t = row t = TMEM lane t)
 //   warps 4-7  softmax warpgroup of tile B
 //   warp  8    TMA producer: both Q tiles once, K tiles through an NK ring
-//              (and, with the gate off, every V tile through the NV ring)
+//              (and, with the gate off or V fetched ahead, every V tile
+//              through the NV ring)
 //   warp  9    MMA issuer (one thread)
-//   warp  10   V issuer (one thread, gate on)
+//   warp  10   V issuer (one thread, gate on, V on demand)
 // TMEM: S_A | S_B | O_A | O_B. P (fp16) is written over the first half of its
 // tile's S columns and read from TMEM by the PV MMA (A operand in TMEM).
 // The MMA thread alternates between the tiles -- PV_A(t), QK_A(t+1), PV_B(t),
@@ -38,7 +39,10 @@
 // neither keeps t, nothing is loaded. V tiles take the NV slots in load order
 // (the n-th loaded tile uses slot n % NV); the MMA thread, which sees both
 // decisions of every tile, counts the loads the same way, and no barrier phase
-// stands for a tile that was not loaded.
+// stands for a tile that was not loaded. As an opt-in (kMode 2) the gated
+// kernel instead fetches every V tile ahead like the ungated one: decisions
+// and outputs are the same, skipped tiles cost their V traffic, and no PV
+// waits for a V load requested after a vote.
 //
 // Precision: S = Q K^T is bf16 x bf16 -> fp32. PV runs in fp16 x fp16 -> fp32:
 // P is at most 2^8 (lazy-rescale bound) and V is read from an fp16 copy made
@@ -111,12 +115,18 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-template <int D, int BQ, int BK, bool kGate>
+// kMode: 0 = no gate (tau = 0: every legal tile kept, V fetched ahead);
+// 1 = gate, V requested only for tiles a query block keeps (the default);
+// 2 = gate, V of every tile fetched ahead whatever the vote (opt-in: skipped
+// tiles then cost their V traffic, but no V load waits behind a vote).
+template <int D, int BQ, int BK, int kMode>
 __global__ void __launch_bounds__(352, 1)
     mala_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
   using Lay = FwdLayout<D, BK>;
+  constexpr bool kGate = kMode != 0;
+  constexpr bool kPrefetchV = kMode != 1;  // V(t) fetched ahead by the producer into slot t % NV
   constexpr int BM = Lay::BM, QPB = BM / BQ;
   constexpr int NK = Lay::NK, NV = Lay::NV;
   constexpr uint32_t IDESC_QK = idesc_bf16(128, BK, false, false);
@@ -234,19 +244,20 @@ __global__ void __launch_bounds__(352, 1)
           tma_load_4d(&tm_k, &k_full[st], sK + st * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, k_off + kb * BK,
                       bt);
         issued = t + 1;
-        if (!kGate) {  // no gate: every tile is kept (load t is tile t), so V(t) is fetched ahead into slot t % NV
+        if (kPrefetchV) {  // every tile is loaded (load t is tile t): V(t) is fetched ahead into slot t % NV
           const int vs = t % NV;
           if (t >= NV && !mbar_wait(&v_empty[vs], ((t / NV) - 1) & 1, fs)) break;
           mbar_arrive_expect_tx(&v_full[vs], Lay::KV_BYTES);
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(&tm_v, &v_full[vs], sV + vs * Lay::KV_BYTES + h * (BK * 128), h * 64, hkv, k_off + kb * BK,
                       bt);
+          if (kGate && p.v_tiles != nullptr) atomicAdd(p.v_tiles, 1ull);
           vissued = t + 1;
         }
       }
       mbar_wait_drain(bar_q, 0);
       for (int t = max(0, issued - NK); t < issued; ++t) mbar_wait_drain(&k_full[t % NK], (t / NK) & 1);
-      if (!kGate)
+      if (kPrefetchV)
         for (int t = max(0, vissued - NV); t < vissued; ++t) mbar_wait_drain(&v_full[t % NV], (t / NV) & 1);
     }
     __syncwarp();
@@ -314,6 +325,12 @@ __global__ void __launch_bounds__(352, 1)
           }
         }
         if (!ok) break;
+        // V fetched ahead: tile t's load has landed before its slot is handed back,
+        // whether or not a PV read it
+        if (kPrefetchV && !v_waited) {
+          if (!mbar_wait(&v_full[vslot], (nload / NV) & 1, fs)) break;
+          v_waited = true;
+        }
         if (v_waited) {
           umma_commit(&v_empty[vslot]);  // V(t) read by both PVs
           ++nload;
@@ -324,7 +341,7 @@ __global__ void __launch_bounds__(352, 1)
     __syncwarp();
   } else if (warp == 10) {
     // ------------------------------------------------------------ V issuer
-    if (kGate && lane == 0) {
+    if (kGate && !kPrefetchV && lane == 0) {
       // the vote of warpgroup x on tile t (bit 0 keep, bit 1 abort), once posted;
       // a bounded wait like every other
       auto vote_of = [&](int x, int t) -> uint32_t {
@@ -440,7 +457,7 @@ __global__ void __launch_bounds__(352, 1)
       const bool my_keep = qi == 0 ? bk0 : bk1;
       const bool need_pv = bk0 || bk1;
       if (tid == 0) {
-        if (kGate) {  // post the vote to the V issuer
+        if (kGate && !kPrefetchV) {  // post the vote to the V issuer
           reinterpret_cast<volatile uint32_t*>(vflag)[x * kVoteRing + t % kVoteRing] =
               (need_pv ? 1u : 0u) | (any_abort ? 2u : 0u);
           __threadfence_block();

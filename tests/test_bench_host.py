@@ -125,3 +125,20 @@ def test_both_arms_report_the_same_config():
     from workloads import C2
     a = bench.bench_config(C2, 1.0, 1)
     assert a == bench.bench_config(C2, 1.0, 1) and a["workload"] == C2.name and a["tau"] == 1.0
+
+
+def test_pair_v_tiles_counts_key_tiles_some_block_of_a_pair_keeps():
+    # brute force over CTAs: a pair of 128-row query tiles (256 rows) loads a
+    # key tile's V once if any of its query blocks keeps that tile
+    rng = np.random.default_rng(5)
+    for L, Bq in ((1000, 128), (777, 64), (300, 64)):
+        nq, nk = -(-L // Bq), -(-L // 128)
+        km = rng.choice(np.array([0, 1, 255], dtype=np.uint8), size=(2, 3, nq, nk))
+        want = 0
+        for b in range(2):
+            for h in range(3):
+                for r0 in range(0, L, 256):
+                    blocks = [qb for qb in range(nq) if r0 <= qb * Bq < r0 + 256]
+                    for kb in range(nk):
+                        want += int(any(km[b, h, qb, kb] == 1 for qb in blocks))
+        assert bench.pair_v_tiles(km, L, Bq) == want

@@ -25,11 +25,11 @@ def _to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def run_fwd_case(mala, w, tau, L=None):
+def run_fwd_case(mala, w, tau, L=None, prefetch_v=False):
     L = w.L if L is None else L
     inp = make_train_inputs(w, L=L)
     q, k, v = (_to_dev(inp[x]) for x in ("q", "k", "v"))
-    o, lse, kept, km = mala.forward(q, k, v, w.scale, tau, w.Bq, w.Bk, keep_map=True)
+    o, lse, kept, km = mala.forward(q, k, v, w.scale, tau, w.Bq, w.Bk, keep_map=True, prefetch_v=prefetch_v)
     assert mala.mala_check_status() == 0
     torch.cuda.synchronize()
     qf, kf, vf = (bf16_bits_to_f64(inp[x]) for x in ("q", "k", "v"))
@@ -47,10 +47,12 @@ def run_fwd_case(mala, w, tau, L=None):
     assert e_lse <= LSE_ABS, e_lse
     if tau == 0:
         assert (km_h == 1).sum() == (ref["keep"] == 1).sum()
-    print(f"[fwd parity] L={L} d={w.d} H={w.Hq}/{w.Hkv} Bq={w.Bq} Bk={w.Bk} tau={tau}: o_rel_l2={e_o:.3e} "
+    print(f"[fwd parity{' prefetch_v' if prefetch_v else ''}] L={L} d={w.d} H={w.Hq}/{w.Hkv} Bq={w.Bq} "
+          f"Bk={w.Bk} tau={tau}: o_rel_l2={e_o:.3e} "
           f"lse_abs={e_lse:.3e} tiles={dec['compared']} in_margin={dec['in_margin']} cascaded={dec['cascaded']} "
           f"kept={int(kept_h.sum())}")
-    return {"o_rel_l2": e_o, "lse_abs": e_lse, **{k_: v_ for k_, v_ in dec.items() if k_ != "diverged_blocks"}}
+    return {"o_rel_l2": e_o, "lse_abs": e_lse, "o": o, "lse": lse, "kept": kept, "km": km,
+            **{k_: v_ for k_, v_ in dec.items() if k_ != "diverged_blocks"}}
 
 
 @pytest.mark.parametrize("tau", [0.0, 1.0])
@@ -133,3 +135,54 @@ def test_fwd_loads_v_only_for_kept_tiles(cuda_lib, tau, Bq):
     print(f"[fwd V tiles] tau={tau} Bq={Bq}: loaded {loaded} of {visits} walked")
     if tau >= 16:
         assert loaded < 0.9 * visits
+
+
+@pytest.mark.parametrize("L,d,Hq,Hkv,Bq,Bk,tau", [
+    (1000, 128, 4, 2, 128, 128, 1.0),  # ragged, GQA
+    (777, 64, 2, 1, 64, 64, 1.0),
+    (1000, 128, 4, 2, 64, 128, 4.0),   # many skips, two query blocks per tile
+    (513, 64, 2, 2, 128, 64, 16.0),
+])
+def test_fwd_prefetch_v_same_results(cuda_lib, L, d, Hq, Hkv, Bq, Bk, tau):
+    """mala_fwd_ex with MALA_FWD_PREFETCH_V: V of every tile fetched ahead of the
+    vote. Decisions and arithmetic are those of the default path, so the outputs
+    match the oracle and equal the default path's bit for bit."""
+    w = TrainWorkload("prefetch", 1, Hq, Hkv, L, d, Bq, Bk, seed=3400 + L + Bq)
+    a = run_fwd_case(cuda_lib, w, tau, prefetch_v=True)
+    b = run_fwd_case(cuda_lib, w, tau, prefetch_v=False)
+    for name in ("o", "lse", "kept", "km"):
+        assert torch.equal(a[name], b[name]), name
+
+
+def test_fwd_prefetch_v_loads_every_tile(cuda_lib):
+    mala = cuda_lib
+    L = 2048
+    w = TrainWorkload("vtiles", 1, 4, 2, L, 128, 128, 128, seed=3300)
+    inp = make_train_inputs(w)
+    q, k, v = (_to_dev(inp[x]) for x in ("q", "k", "v"))
+    counter = torch.zeros(1, dtype=torch.int64, device="cuda")
+    assert mala.mala_test_hooks(0, -1, counter) == 0
+    try:
+        _, _, _, km = mala.forward(q, k, v, w.scale, 16.0, w.Bq, w.Bk, keep_map=True, prefetch_v=True)
+        assert mala.mala_check_status() == 0
+    finally:
+        mala.mala_test_hooks(0, -1, None)
+    visits = w.B * w.Hq * sum((min(pr * 256 + 256, L) - 1) // w.Bk + 1 for pr in range(-(-L // 256)))
+    assert int(counter.item()) == visits
+    assert pair_v_tiles(km.cpu().numpy(), L, w.Bq) < 0.9 * visits  # tau = 16 skips, the V loads do not
+
+
+def test_fwd_ex_rejects_unknown_flags(cuda_lib):
+    mala = cuda_lib
+    L, d = 128, 128  # properly sized buffers, although the flags are checked before anything is read
+    q = torch.zeros((1, L, 1, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 1, L), dtype=torch.float32, device="cuda")
+    kept = torch.empty((1,), dtype=torch.int32, device="cuda")
+    wsb = mala.mala_fwd_workspace_size(1, 1, L, d)
+    ws = torch.empty((wsb,), dtype=torch.uint8, device="cuda")
+    rc = mala.mala_fwd_ex(q, q, q, o, lse, 1, 1, 1, L, d, 0.1, 1.0, 128, 128, ws, wsb, kept, None, None, flags=2)
+    assert rc == mala.MALA_ERR_INVALID_ARG
+    rc = mala.mala_fwd_ex(q, q, q, o, lse, 1, 1, 1, L, d, 0.1, 1.0, 128, 128, ws, wsb, kept, None, None,
+                          flags=mala.MALA_FWD_PREFETCH_V)
+    assert rc == mala.MALA_OK and mala.mala_check_status() == 0
