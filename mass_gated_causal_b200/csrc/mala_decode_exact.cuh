@@ -56,14 +56,17 @@ struct DxParams {
 };
 
 // Shared-memory layout of the PV kernel: an NS-stage ring of
-// [D/64][BK][64] bf16 tiles (128-byte swizzle, as the TMA writes them), a
+// [D/64][BK][64] bf16 tiles (128-byte swizzle, as the TMA writes them) with
+// the tile's scores of the group's heads ([GP][BK] fp32 per stage), a
 // [2][GP][BK] fp32 tile and the ring's barriers.
 template <int D, int BK, int GP>
 struct DxLayout {
   static constexpr int NS = 4;
   static constexpr int TB = BK * D * 2;
+  static constexpr int SB = GP * BK * 4;                  // scores of one stage
   static constexpr int OFF_RING = 0;
-  static constexpr int OFF_T = OFF_RING + NS * TB;        // fp32 [2][GP][BK]: P by tile parity
+  static constexpr int OFF_SC = OFF_RING + NS * TB;       // fp32 [NS][GP][BK]: the stages' scores
+  static constexpr int OFF_T = OFF_SC + NS * SB;          // fp32 [2][GP][BK]: P by tile parity
   static constexpr int OFF_O = OFF_T + 2 * GP * BK * 4;   // fp32 [8][GP][D + 4] (PV reduction)
   static constexpr int OFF_LIST = OFF_O + 8 * GP * (D + 4) * 4;  // int tiles [LIST], uint8 bits [LIST]
   static constexpr int LIST = 1024;
@@ -86,7 +89,7 @@ __device__ __forceinline__ uint32_t dx_row_chunk(uint32_t base, int j, int cc) {
 // rows per step (fully used lines); the G partial dot products are summed over
 // the 16 lanes by a reduce-scatter, after which lane c owns head c / (16 / GP).
 template <int D, int BK, int GP>
-__global__ void __launch_bounds__(256) mala_dx_scores_kernel(const DxParams p) {
+__global__ void __launch_bounds__(256, 2) mala_dx_scores_kernel(const DxParams p) {
   constexpr int CPL = D / 16;  // columns per lane
   constexpr int LPH = 16 / GP; // lanes per head after the reduce-scatter
   __shared__ float sS[8][GP][BK];
@@ -107,7 +110,11 @@ __global__ void __launch_bounds__(256) mala_dx_scores_kernel(const DxParams p) {
       qf[g][e] = g < p.G ? bf16lo_to_f32(p.q[(static_cast<size_t>(b) * p.Hq + hq0 + g) * D + c * CPL + e]) : 0.f;
   const uint16_t* krow0 = p.kc + (static_cast<size_t>(b) * p.Lk * p.Hkv + hkv) * D + c * CPL;
   const size_t kstride = static_cast<size_t>(p.Hkv) * D;
-  constexpr int UNR = 4;  // rows per lane and group; the next group's loads are issued before this one is used
+  // rows per lane and group; the next group's loads are issued before this one
+  // is used. Eight (4 KB in flight per warp, two CTAs per SM at 128 registers)
+  // measured 3% faster over the whole decode than four (three CTAs per SM);
+  // sixteen (one CTA per SM) and eight at three CTAs per SM (spills) were slower.
+  constexpr int UNR = 8;
   uint32_t nxt[UNR][CPL / 2];
   auto load_group = [&](int it0) {
 #pragma unroll
@@ -245,9 +252,10 @@ __global__ void __launch_bounds__(128) mala_dx_scan_kernel(const DxParams p) {
 // largest M_t of its kept tiles and its normaliser l = sum over those tiles of
 // 2^{L_t - m} (both from the per-tile pairs). Warp 8 lists the tiles some head
 // of the group keeps (with a bit per head) and streams their V by TMA through
-// the ring; a tile no head keeps is never read. Per listed tile the compute
-// warps form P = 2^{s - m} (0 for a head that skips the tile; the scores of
-// the next tile are loaded while this one is used) in shared memory, and warp
+// the ring, together with the tile's scores of the group's heads (bulk copies
+// on the same barrier, so no compute warp waits on a global load); a tile no
+// head keeps is never read. Per listed tile the compute warps form
+// P = 2^{s - m} (0 for a head that skips the tile) in shared memory, and warp
 // w takes keys [BK/8 * w, BK/8 * (w+1)), two per step: lane c of half h
 // accumulates D/16 columns of the G heads' P V over its rows.
 template <int D, int BK, int GP>
@@ -261,6 +269,7 @@ __global__ void __launch_bounds__(288, 1) mala_dx_pv_kernel(const __grid_constan
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* sP = reinterpret_cast<float*>(smem + Lay::OFF_T);  // [2][GP][BK]
+  const float* sSc = reinterpret_cast<const float*>(smem + Lay::OFF_SC);  // [NS][GP][BK]
   float* sO = reinterpret_cast<float*>(smem + Lay::OFF_O);  // [8][GP][D + 4]
   int* sList = reinterpret_cast<int*>(smem + Lay::OFF_LIST);
   uint8_t* sBits = smem + Lay::OFF_LIST + LIST * 4;
@@ -338,37 +347,32 @@ __global__ void __launch_bounds__(288, 1) mala_dx_pv_kernel(const __grid_constan
         for (int i = 0; i < n; ++i) {
           const int ig = base + i, st = ig % NS;
           if (ig >= NS && !mbar_wait(&empty[st], ((ig / NS) - 1) & 1, fs)) break;
-          mbar_arrive_expect_tx(&full[st], TB);
+          mbar_arrive_expect_tx(&full[st], TB + p.G * BK * 4);
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(&tm_v, &full[st], smem + Lay::OFF_RING + st * TB + h * (BK * 128), h * 64, hkv,
                         sList[i] * BK, b);
+          // the scores rows start on 512-byte boundaries (rows of Lkp = nk * BK floats, tiles of BK)
+          for (int g = 0; g < p.G; ++g)
+            bulk_load_1d(smem + Lay::OFF_SC + (st * GP + g) * BK * 4,
+                         p.scores + (r0 + g) * p.Lkp + static_cast<size_t>(sList[i]) * BK, BK * 4, &full[st]);
           issued = ig + 1;
         }
       }
     } else {
-      float scn[NPT];  // the scores of tile i + 1, loaded while tile i is used
-      auto load_scores = [&](int i) {
-        const int kb = sList[i];
-#pragma unroll
-        for (int k = 0; k < NPT; ++k) {
-          const int idx = tid + k * 256, g = idx / BK, j = idx % BK;
-          scn[k] = (idx < GP * BK && ((sBits[i] >> g) & 1u))
-                       ? __ldg(p.scores + (r0 + g) * p.Lkp + static_cast<size_t>(kb) * BK + j)
-                       : -INFINITY;
-        }
-      };
-      if (n > 0) load_scores(0);
       for (int i = 0; i < n; ++i) {
         const int ig = base + i, st = ig % NS;
         float* P = sP + (ig & 1) * GP * BK;
+        const bool ok = mbar_wait_warp(&full[st], (ig / NS) & 1, fs);  // V and the scores of this tile
+        const uint32_t bits = sBits[i];
 #pragma unroll
         for (int k = 0; k < NPT; ++k) {
-          const int idx = tid + k * 256;
-          if (idx < GP * BK) P[idx] = scn[k] == -INFINITY ? 0.f : ex2_approx(scn[k] - sM[idx / BK]);
+          const int idx = tid + k * 256, g = idx / BK;
+          if (idx < GP * BK) {
+            const float s = (ok && ((bits >> g) & 1u)) ? sSc[st * GP * BK + idx] : -INFINITY;
+            P[idx] = s == -INFINITY ? 0.f : ex2_approx(s - sM[g]);
+          }
         }
-        if (i + 1 < n) load_scores(i + 1);
         named_bar_sync(1, 256);  // P of this tile is in place (and the one two tiles back is read)
-        const bool ok = mbar_wait_warp(&full[st], (ig / NS) & 1, fs);
         if (ok) {
 #pragma unroll
           for (int u = 0; u < KPW / 2; ++u) {
