@@ -90,6 +90,13 @@ def packed_flops(lens, Hq, d, Bq, Bk, keep_f, keep_b):
     return fl
 
 
+def walked_key_tiles(B: int, Hq: int, L: int, Bk: int) -> int:
+    """Key tiles the forward's CTAs walk in a training forward: each CTA owns a
+    pair of 128-row query tiles of one (b, hq) and visits key tiles 0 .. the
+    tile of the pair's last row."""
+    return B * Hq * sum((min(pr * 256 + 256, L) - 1) // Bk + 1 for pr in range(-(-L // 256)))
+
+
 def pair_v_tiles(km, L: int, Bq: int) -> int:
     """V tiles the default forward loads: a CTA owns a pair of 128-row query
     tiles of one (b, hq) and loads a key tile's V once if some query block of
@@ -380,7 +387,7 @@ def run_cuda(args):
         return fn
 
     prefetch = {}
-    walked = B * Hq * sum((min(pr * 256 + 256, L) - 1) // w.Bk + 1 for pr in range(-(-L // 256)))
+    walked = walked_key_tiles(B, Hq, L, w.Bk)
     for tau_p in sorted(km_by_tau):
         t_dem, _, _ = timed(fwd_only(tau_p, 0), 5, 3)
         t_pre, _, _ = timed(fwd_only(tau_p, mala.MALA_FWD_PREFETCH_V), 5, 3)

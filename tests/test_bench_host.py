@@ -142,3 +142,14 @@ def test_pair_v_tiles_counts_key_tiles_some_block_of_a_pair_keeps():
                     for kb in range(nk):
                         want += int(any(km[b, h, qb, kb] == 1 for qb in blocks))
         assert bench.pair_v_tiles(km, L, Bq) == want
+
+
+def test_walked_key_tiles_brute_force():
+    # every (b, hq, pair of 128-row tiles) walks the key tiles up to the one
+    # holding its last row's key: the union over the pair's rows of the causal range
+    for L, Bk in ((1, 128), (128, 64), (1000, 128), (777, 64), (4096, 128)):
+        want = 0
+        for r0 in range(0, L, 256):
+            last = min(r0 + 256, L) - 1
+            want += len({k // Bk for k in range(last + 1)})
+        assert bench.walked_key_tiles(2, 3, L, Bk) == 6 * want
